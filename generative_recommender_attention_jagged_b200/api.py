@@ -1,0 +1,177 @@
+"""Python entry points over libhstu.so, with the same names as the C ABI.
+
+Tensors are torch CUDA tensors (torch provides device memory and the current
+stream); everything else is the library's.  Inputs on the CPU are refused.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float32: _lib.DT_F32, torch.bfloat16: _lib.DT_BF16}
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(name: str, t: Optional[torch.Tensor], dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _rows_view(name: str, t: torch.Tensor, H: int, d: int) -> int:
+    """Token stride (elements) of a [T,H,d] (or [T,H*d]) view with packed heads."""
+    if t.dim() == 3:
+        ok = t.stride(2) == 1 and t.stride(1) == d
+    else:
+        ok = t.stride(1) == 1
+    if not ok:
+        raise ValueError(f"{name}: heads and features must be packed (stride 1 / d)")
+    return t.stride(0) if t.shape[0] > 1 else H * d
+
+
+def attn_params(*, batch: int, num_heads: int, head_dim: int, n_max: int, total_tokens: int,
+                max_seq_len: int, dtype: torch.dtype, alpha: Optional[float] = None,
+                num_ts_buckets: int = 128, qkv_stride: int = 0, u_stride: int = 0,
+                ln_eps: float = 1e-5, flags: int = 0) -> _lib.AttnParams:
+    return _lib.AttnParams(batch=batch, num_heads=num_heads, head_dim=head_dim, n_max=n_max,
+                           num_ts_buckets=num_ts_buckets, total_tokens=total_tokens,
+                           max_seq_len=max_seq_len, qkv_stride=qkv_stride, u_stride=u_stride,
+                           alpha=(1.0 / math.sqrt(head_dim)) if alpha is None else alpha,
+                           ln_eps=ln_eps, dtype=_DT[dtype], flags=flags)
+
+
+def hstu_attn_workspace_size(p: _lib.AttnParams) -> int:
+    return int(_lib.load().hstu_attn_workspace_size(ctypes.byref(p)))
+
+
+def hstu_attn_paged_workspace_size(p: _lib.AttnParams, num_splits: int) -> int:
+    return int(_lib.load().hstu_attn_paged_workspace_size(ctypes.byref(p), num_splits))
+
+
+def hstu_attn_paged_default_splits(p: _lib.AttnParams, max_cached_len: int) -> int:
+    return int(_lib.load().hstu_attn_paged_default_splits(ctypes.byref(p), max_cached_len))
+
+
+def hstu_attn_fwd(q, k, v, u, seq_offsets, timestamps, rab_pos, rab_ts, *, n_max: int,
+                  alpha: Optional[float] = None, num_candidates=None, ln_gamma=None, ln_beta=None,
+                  ln_eps: float = 1e-5, max_seq_len: Optional[int] = None, out=None,
+                  workspace=None, raw_av: bool = False, force_simt: bool = False, stages: int = 0,
+                  stream=None, params: Optional[_lib.AttnParams] = None):
+    """Jagged HSTU attention forward; returns out [T, H*d] (or o [T,H,d] fp32 when raw_av)."""
+    T, H, d = q.shape
+    dt = q.dtype
+    for name, t in (("q", q), ("k", k), ("v", v), ("u", u)):
+        _need_cuda(name, t, dt)
+    _need_cuda("seq_offsets", seq_offsets, torch.int32)
+    _need_cuda("timestamps", timestamps, torch.int64)
+    _need_cuda("num_candidates", num_candidates, torch.int32)
+    for name, t in (("rab_pos", rab_pos), ("rab_ts", rab_ts), ("ln_gamma", ln_gamma), ("ln_beta", ln_beta)):
+        _need_cuda(name, t, torch.float32)
+    qs = _rows_view("q", q, H, d)
+    if _rows_view("k", k, H, d) != qs or _rows_view("v", v, H, d) != qs:
+        raise ValueError("q, k and v must share one token stride")
+    us = _rows_view("u", u, H, d)
+    B = seq_offsets.numel() - 1
+    flags = (_lib.F_OUTPUT_RAW_AV if raw_av else 0) | (_lib.F_FORCE_SIMT if force_simt else 0) | stages
+    if params is None:
+        params = attn_params(batch=B, num_heads=H, head_dim=d, n_max=n_max, total_tokens=T,
+                             max_seq_len=n_max if max_seq_len is None else max_seq_len, dtype=dt,
+                             alpha=alpha, num_ts_buckets=rab_ts.numel(), qkv_stride=qs, u_stride=us,
+                             ln_eps=ln_eps, flags=flags)
+    if out is None:
+        out = (torch.empty(T, H, d, dtype=torch.float32, device=q.device) if raw_av
+               else torch.empty(T, H * d, dtype=dt, device=q.device))
+    if workspace is None:
+        workspace = torch.empty(hstu_attn_workspace_size(params), dtype=torch.uint8, device=q.device)
+    rc = _lib.load().hstu_attn_fwd(ctypes.byref(params), _p(q), _p(k), _p(v), _p(u), _p(seq_offsets),
+                                   _p(timestamps), _p(num_candidates), _p(rab_pos), _p(rab_ts),
+                                   _p(ln_gamma), _p(ln_beta), _p(out), _p(workspace),
+                                   workspace.numel(), _stream(stream))
+    _lib.check(rc, "hstu_attn_fwd")
+    return out
+
+
+def hstu_attn_fwd_paged(q, k, v, u, new_offsets, timestamps, ts_offsets, rab_pos, rab_ts, k_pool,
+                        v_pool, kv_page_table, cached_lens, *, n_max: int, alpha: Optional[float] = None,
+                        num_candidates=None, ln_gamma=None, ln_beta=None, ln_eps: float = 1e-5,
+                        max_seq_len: Optional[int] = None, num_splits: Optional[int] = None,
+                        max_cached_len: Optional[int] = None, out=None, workspace=None,
+                        raw_av: bool = False, force_simt: bool = False, stages: int = 0, stream=None):
+    """Incremental HSTU attention of new tokens over a paged K/V prefix."""
+    T, H, d = q.shape
+    dt = q.dtype
+    for name, t in (("q", q), ("k", k), ("v", v), ("u", u), ("k_pool", k_pool), ("v_pool", v_pool)):
+        _need_cuda(name, t, dt)
+    for name, t in (("new_offsets", new_offsets), ("ts_offsets", ts_offsets),
+                    ("kv_page_table", kv_page_table), ("cached_lens", cached_lens),
+                    ("num_candidates", num_candidates)):
+        _need_cuda(name, t, torch.int32)
+    _need_cuda("timestamps", timestamps, torch.int64)
+    if not (k_pool.is_contiguous() and v_pool.is_contiguous() and kv_page_table.is_contiguous()):
+        raise ValueError("k_pool, v_pool and kv_page_table must be contiguous")
+    num_pages, _, page_size, _ = k_pool.shape
+    qs = _rows_view("q", q, H, d)
+    if _rows_view("k", k, H, d) != qs or _rows_view("v", v, H, d) != qs:
+        raise ValueError("q, k and v must share one token stride")
+    us = _rows_view("u", u, H, d)
+    B = new_offsets.numel() - 1
+    flags = (_lib.F_OUTPUT_RAW_AV if raw_av else 0) | (_lib.F_FORCE_SIMT if force_simt else 0) | stages
+    params = attn_params(batch=B, num_heads=H, head_dim=d, n_max=n_max, total_tokens=T,
+                         max_seq_len=n_max if max_seq_len is None else max_seq_len, dtype=dt,
+                         alpha=alpha, num_ts_buckets=rab_ts.numel(), qkv_stride=qs, u_stride=us,
+                         ln_eps=ln_eps, flags=flags)
+    if num_splits is None:
+        mc = n_max if max_cached_len is None else max_cached_len
+        num_splits = hstu_attn_paged_default_splits(params, mc)
+    if out is None:
+        out = (torch.empty(T, H, d, dtype=torch.float32, device=q.device) if raw_av
+               else torch.empty(T, H * d, dtype=dt, device=q.device))
+    if workspace is None:
+        workspace = torch.empty(hstu_attn_paged_workspace_size(params, num_splits), dtype=torch.uint8,
+                                device=q.device)
+    rc = _lib.load().hstu_attn_fwd_paged(
+        ctypes.byref(params), _p(q), _p(k), _p(v), _p(u), _p(new_offsets), _p(timestamps), _p(ts_offsets),
+        _p(num_candidates), _p(rab_pos), _p(rab_ts), _p(ln_gamma), _p(ln_beta), _p(k_pool), _p(v_pool),
+        num_pages, _p(kv_page_table), kv_page_table.shape[1], page_size, _p(cached_lens), num_splits,
+        _p(out), _p(workspace), workspace.numel(), _stream(stream))
+    _lib.check(rc, "hstu_attn_fwd_paged")
+    return out
+
+
+def hstu_ts_bucket(dt: torch.Tensor, num_buckets: int = 128, out=None, stream=None) -> torch.Tensor:
+    _need_cuda("dt", dt, torch.int64)
+    dt = dt.contiguous()
+    if out is None:
+        out = torch.empty(dt.shape, dtype=torch.int32, device=dt.device)
+    rc = _lib.load().hstu_ts_bucket(_p(dt), dt.numel(), num_buckets, _p(out), _stream(stream))
+    _lib.check(rc, "hstu_ts_bucket")
+    return out
+
+
+def hstu_check_device_error(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns the device status word of `workspace`."""
+    return int(_lib.load().hstu_check_device_error(_p(workspace), _stream(stream)))
+
+
+def hstu_status_string(status: int) -> str:
+    return _lib.load().hstu_status_string(status).decode()
+
+
+def hstu_version() -> int:
+    return int(_lib.load().hstu_version())

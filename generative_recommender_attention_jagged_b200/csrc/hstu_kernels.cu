@@ -1,0 +1,406 @@
+// Validation, tile scheduling, the CUDA-core attention kernel, the fused
+// LayerNorm(A.V) * U epilogue and the time-bucket kernel.
+//
+// The attention definition these kernels follow is the one written in
+// include/hstu.h (from "Generative Recommenders at Scale", Inside NVIDIA's
+// GPU-native stack; "How Generative Recommenders Are Redefining RecSys at
+// Scale", Takeaways; "HSTU Generative Recommenders: Deploy on GPU Cloud",
+// M-FALCON section).
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "device_common.cuh"
+
+namespace hstu {
+
+namespace {
+
+constexpr long long kTsLimit = 1ll << 61;  // |timestamp| bound that keeps t_i + 1 - thr in range
+
+// ---------------------------------------------------------------------------
+// validate: one block per user
+// ---------------------------------------------------------------------------
+__global__ void validate_kernel(const AttnArgs a) {
+  const int u = blockIdx.x;
+  __shared__ int s_ok;
+  __shared__ int s_n, s_tso, s_pages;
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const int q0 = a.q_offsets[u], q1 = a.q_offsets[u + 1];
+    if (u == 0 && q0 != 0) ok = 0;
+    if (u == a.B - 1 && q1 != a.T_q) ok = 0;
+    if (q0 < 0 || q1 < q0 || q1 > a.T_q) ok = 0;
+    const int L = a.paged ? a.cached_lens[u] : 0;
+    if (L < 0) ok = 0;
+    const long long n = (long long)L + (q1 - q0);
+    if (n > a.n_max) ok = 0;
+    const int c = a.num_cand ? a.num_cand[u] : 0;
+    if (c < 0 || c > q1 - q0) ok = 0;
+    int tso = q0, pages = 0;
+    if (a.paged) {
+      tso = a.ts_offsets[u];
+      if (u == 0 && tso != 0) ok = 0;
+      if ((long long)a.ts_offsets[u + 1] - tso != n) ok = 0;
+      pages = ceil_div(L, a.page_size);
+      if (pages > a.max_pages) ok = 0;
+    }
+    if (!ok) report_error(a.hdr, kErrLength, u);
+    s_ok = ok;
+    s_n = (int)n;
+    s_tso = tso;
+    s_pages = pages;
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  if (a.paged) {
+    for (int x = threadIdx.x; x < s_pages; x += blockDim.x) {
+      const int pid = a.page_table[(size_t)u * a.max_pages + x];
+      if (pid < 0 || pid >= a.num_pages) report_error(a.hdr, kErrPage, u);
+    }
+  }
+  const int64_t* ts = a.ts + s_tso;
+  for (int j = threadIdx.x; j < s_n; j += blockDim.x) {
+    const long long t = ts[j];
+    if (t > kTsLimit || t < -kTsLimit || (j > 0 && t < ts[j - 1])) report_error(a.hdr, kErrUnsorted, u);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// schedule: one block builds the work list, longest query tiles first
+// ---------------------------------------------------------------------------
+constexpr int kSchedThreads = 1024;
+constexpr int kCostBins = 1024;
+
+__global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const AttnArgs a) {
+  __shared__ int hist[kCostBins];
+  __shared__ int start[kCostBins];
+  __shared__ int s_status;
+  const int tid = threadIdx.x;
+  for (int x = tid; x < kCostBins; x += blockDim.x) hist[x] = 0;
+  if (tid == 0) s_status = a.hdr->status;
+  __syncthreads();
+  if (s_status != 0) {
+    if (tid == 0) a.hdr->n_items = 0;
+    return;
+  }
+  const int per = a.H * a.num_splits;
+  auto cost_of = [&](int user, int m) {
+    const TileGeom g = tile_geom(a, user, m);
+    const int c = ceil_div(g.n_tiles, a.num_splits);
+    return min(c, kCostBins - 1);
+  };
+  for (int u = tid; u < a.B; u += blockDim.x) {
+    const int nq = a.q_offsets[u + 1] - a.q_offsets[u];
+    for (int m = ceil_div(nq, kTile) - 1; m >= 0; --m) atomicAdd(&hist[cost_of(u, m)], per);
+  }
+  __syncthreads();
+  // start[c] = number of items with a cost above c (descending order)
+  if (tid < 32) {
+    int carry = 0;
+    for (int base = kCostBins - 32; base >= 0; base -= 32) {
+      const int c = base + 31 - tid;  // lane 0 takes the highest cost of the chunk
+      const int v = hist[c];
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(~0u, incl, o);
+        if (tid >= o) incl += y;
+      }
+      start[c] = carry + incl - v;
+      carry += __shfl_sync(~0u, incl, 31);
+    }
+    if (tid == 0) a.hdr->n_items = min(carry, a.max_items);
+  }
+  __syncthreads();
+  for (int u = tid; u < a.B; u += blockDim.x) {
+    const int nq = a.q_offsets[u + 1] - a.q_offsets[u];
+    for (int m = ceil_div(nq, kTile) - 1; m >= 0; --m) {
+      const int pos = atomicAdd(&start[cost_of(u, m)], per);
+      for (int h = 0; h < a.H; ++h)
+        for (int s = 0; s < a.num_splits; ++s) {
+          const int idx = pos + h * a.num_splits + s;
+          if (idx < a.max_items) a.items[idx] = WorkItem{u, m, h, s};
+        }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core attention: one warp per (query row, head); any d <= 256, fp32 or
+// bf16 inputs; jagged or paged keys.  Writes the unscaled sum
+// sum_j SiLU(s_ij) v_j (self term of candidates included) to o_ws.
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+constexpr int kSimtMaxPerLane = 8;  // d <= 256
+
+__device__ __forceinline__ int find_user(const int32_t* off, int B, int row) {
+  int lo = 0, hi = B - 1;  // largest u with off[u] <= row
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= row) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) attn_simt_kernel(const AttnArgs a, const BucketTable tab) {
+  __shared__ long long thr[kMaxBuckets];
+  for (int x = threadIdx.x; x < kMaxBuckets; x += blockDim.x) thr[x] = tab.thr[x];
+  __syncthreads();
+  if (a.hdr->status != 0) return;
+  const int lane = threadIdx.x & 31;
+  const int warps_per_block = blockDim.x >> 5;
+  const long long total = (long long)a.T_q * a.H;
+  const T* q = static_cast<const T*>(a.q);
+  const T* k = static_cast<const T*>(a.k);
+  const T* v = static_cast<const T*>(a.v);
+  const T* kp = static_cast<const T*>(a.k_pool);
+  const T* vp = static_cast<const T*>(a.v_pool);
+  const int d = a.d;
+  const int per_lane = (d + 31) >> 5;
+  for (long long w = (long long)blockIdx.x * warps_per_block + (threadIdx.x >> 5); w < total;
+       w += (long long)gridDim.x * warps_per_block) {
+    const int row = (int)(w / a.H);
+    const int head = (int)(w % a.H);
+    const int u = find_user(a.q_offsets, a.B, row);
+    const int q0 = a.q_offsets[u];
+    const int L = a.paged ? a.cached_lens[u] : 0;
+    const int n = L + (a.q_offsets[u + 1] - q0);
+    const int hist = n - (a.num_cand ? a.num_cand[u] : 0);
+    const int tso = a.paged ? a.ts_offsets[u] : q0;
+    const int i = L + (row - q0);
+    const long long t_i = a.ts[tso + i];
+    const int p_i = min(i, hist);
+    float qv[kSimtMaxPerLane], acc[kSimtMaxPerLane];
+#pragma unroll
+    for (int x = 0; x < kSimtMaxPerLane; ++x) {
+      const int e = lane + 32 * x;
+      qv[x] = (x < per_lane && e < d) ? to_f(q[(size_t)row * a.qkv_stride + head * d + e]) : 0.f;
+      acc[x] = 0.f;
+    }
+    // allowed keys: [0, i] for history rows; [0, hist) and i for candidates
+    const int j_end = i < hist ? i + 1 : hist;
+    for (int jj = 0; jj <= j_end; ++jj) {
+      int j = jj;
+      if (jj == j_end) {
+        if (i < hist) break;  // history rows: the loop already covered j = i
+        j = i;                // candidate self term
+      }
+      const T* kr;
+      const T* vr;
+      if (j < L) {
+        const int pid = a.page_table[(size_t)u * a.max_pages + j / a.page_size];
+        const size_t base = (((size_t)pid * a.H + head) * a.page_size + (j % a.page_size)) * d;
+        kr = kp + base;
+        vr = vp + base;
+      } else {
+        const size_t base = (size_t)(q0 + j - L) * a.qkv_stride + head * d;
+        kr = k + base;
+        vr = v + base;
+      }
+      float part = 0.f;
+#pragma unroll
+      for (int x = 0; x < kSimtMaxPerLane; ++x) {
+        const int e = lane + 32 * x;
+        if (x < per_lane && e < d) part = fmaf(qv[x], to_f(kr[e]), part);
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(~0u, part, o);
+      const int p_j = min(j, hist);
+      const int bkt = bucket_of_dt(thr, t_i - a.ts[tso + j]);
+      const float s = a.alpha * part + a.rab_pos[p_i - p_j + a.n_max - 1] + a.rab_ts[bkt];
+      const float wgt = s / (1.f + expf(-s));
+#pragma unroll
+      for (int x = 0; x < kSimtMaxPerLane; ++x) {
+        const int e = lane + 32 * x;
+        if (x < per_lane && e < d) acc[x] = fmaf(wgt, to_f(vr[e]), acc[x]);
+      }
+    }
+    float* orow = a.o_ws + ((size_t)row * a.H + head) * d;
+#pragma unroll
+    for (int x = 0; x < kSimtMaxPerLane; ++x) {
+      const int e = lane + 32 * x;
+      if (x < per_lane && e < d) orow[e] = acc[x];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue: one warp per token.  o = (sum of split partials [+ candidate self
+// term]) / N_max; y = (LayerNorm(o) * gamma + beta) * u over the H*d features
+// with warp-shuffle reductions.  D = H*d <= 1024.
+// ---------------------------------------------------------------------------
+constexpr int kEpiMax = 32;  // values per lane: D <= 1024
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(~0u, x, o);
+  return x;
+}
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(256) epilogue_kernel(const AttnArgs a) {
+  if (a.hdr->status != 0) return;
+  const int lane = threadIdx.x & 31;
+  const int warps_per_block = blockDim.x >> 5;
+  const int D = a.H * a.d;
+  const int per_lane = (D + 31) >> 5;
+  const float inv_n = 1.0f / (float)a.n_max;
+  const TIn* uu = static_cast<const TIn*>(a.u);
+  const TIn* q = static_cast<const TIn*>(a.q);
+  const TIn* k = static_cast<const TIn*>(a.k);
+  const TIn* v = static_cast<const TIn*>(a.v);
+  const size_t split_stride = (size_t)a.T_q * D;
+  for (int row = blockIdx.x * warps_per_block + (threadIdx.x >> 5); row < a.T_q;
+       row += gridDim.x * warps_per_block) {
+    float o[kEpiMax];
+#pragma unroll
+    for (int x = 0; x < kEpiMax; ++x) {
+      const int e = lane + 32 * x;
+      float s = 0.f;
+      if (x < per_lane && e < D) {
+        const float* src = a.o_ws + (size_t)row * D + e;
+        for (int sp = 0; sp < a.num_splits; ++sp) s += src[sp * split_stride];
+      }
+      o[x] = s;
+    }
+    if (a.self_term && a.num_cand) {
+      const int u = find_user(a.q_offsets, a.B, row);
+      const int q0 = a.q_offsets[u];
+      const int nq = a.q_offsets[u + 1] - q0;
+      if (row - q0 >= nq - a.num_cand[u]) {
+        const float bias = a.rab_pos[a.n_max - 1] + a.rab_ts[0];
+        for (int h = 0; h < a.H; ++h) {
+          float part = 0.f;
+#pragma unroll
+          for (int x = 0; x < kEpiMax; ++x) {
+            const int e = lane + 32 * x;
+            if (x < per_lane && e < D && e / a.d == h) {
+              const size_t off = (size_t)row * a.qkv_stride + e;
+              part = fmaf(to_f(q[off]), to_f(k[off]), part);
+            }
+          }
+          const float s = a.alpha * warp_sum(part) + bias;
+          const float wgt = s / (1.f + expf(-s));
+#pragma unroll
+          for (int x = 0; x < kEpiMax; ++x) {
+            const int e = lane + 32 * x;
+            if (x < per_lane && e < D && e / a.d == h) o[x] = fmaf(wgt, to_f(v[(size_t)row * a.qkv_stride + e]), o[x]);
+          }
+        }
+      }
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int x = 0; x < kEpiMax; ++x) {
+      o[x] *= inv_n;
+      sum += o[x];  // lanes past D hold 0
+    }
+    if (a.out_raw) {
+      float* out = static_cast<float*>(a.out) + (size_t)row * D;
+#pragma unroll
+      for (int x = 0; x < kEpiMax; ++x) {
+        const int e = lane + 32 * x;
+        if (x < per_lane && e < D) out[e] = o[x];
+      }
+      continue;
+    }
+    const float mean = warp_sum(sum) / (float)D;
+    float sq = 0.f;
+#pragma unroll
+    for (int x = 0; x < kEpiMax; ++x) {
+      const int e = lane + 32 * x;
+      if (x < per_lane && e < D) {
+        const float c = o[x] - mean;
+        sq = fmaf(c, c, sq);
+      }
+    }
+    const float rstd = rsqrtf(warp_sum(sq) / (float)D + a.ln_eps);
+    TOut* out = static_cast<TOut*>(a.out) + (size_t)row * D;
+#pragma unroll
+    for (int x = 0; x < kEpiMax; ++x) {
+      const int e = lane + 32 * x;
+      if (x < per_lane && e < D) {
+        const float g = a.ln_gamma ? a.ln_gamma[e] : 1.f;
+        const float b = a.ln_beta ? a.ln_beta[e] : 0.f;
+        const float y = ((o[x] - mean) * rstd * g + b) * to_f(uu[(size_t)row * a.u_stride + e]);
+        if constexpr (sizeof(TOut) == 2) out[e] = __float2bfloat16_rn(y);
+        else out[e] = y;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// standalone time-bucket kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) ts_bucket_kernel(const int64_t* __restrict__ dt, int64_t n,
+                                                        int32_t* __restrict__ out, const BucketTable tab) {
+  __shared__ long long thr[kMaxBuckets];
+  for (int x = threadIdx.x; x < kMaxBuckets; x += blockDim.x) thr[x] = tab.thr[x];
+  __syncthreads();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = bucket_of_dt(thr, dt[i]);
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_validate(const AttnArgs& a, cudaStream_t s) {
+  validate_kernel<<<a.B, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_schedule(const AttnArgs& a, cudaStream_t s) {
+  schedule_kernel<<<1, kSchedThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_simt(const AttnArgs& a, const BucketTable& thr, cudaStream_t s) {
+  const long long warps = (long long)a.T_q * a.H;
+  const int blocks = (int)std::min<long long>((warps + 7) / 8, (long long)num_sms() * 16);
+  if (a.in_bf16) attn_simt_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(a, thr);
+  else attn_simt_kernel<float><<<blocks, 256, 0, s>>>(a, thr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_epilogue(const AttnArgs& a, cudaStream_t s) {
+  const int blocks = std::max(1, std::min((a.T_q + 7) / 8, num_sms() * 16));
+  if (a.in_bf16) {
+    if (a.out_bf16) epilogue_kernel<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, s>>>(a);
+    else epilogue_kernel<__nv_bfloat16, float><<<blocks, 256, 0, s>>>(a);
+  } else {
+    if (a.out_bf16) epilogue_kernel<float, __nv_bfloat16><<<blocks, 256, 0, s>>>(a);
+    else epilogue_kernel<float, float><<<blocks, 256, 0, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ts_bucket(const int64_t* dt, int64_t n, int32_t* out, const BucketTable& thr,
+                             cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const long long blocks = std::min<long long>((n + 255) / 256, (long long)num_sms() * 8);
+  ts_bucket_kernel<<<(int)blocks, 256, 0, s>>>(dt, n, out, thr);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

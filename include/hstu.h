@@ -1,0 +1,190 @@
+/*
+ * hstu.h - C ABI of libhstu.so: HSTU pointwise attention over jagged
+ * per-user sequences on NVIDIA B200 (sm_100a).
+ *
+ * The operation (one definition for every entry point below):
+ *
+ *   For user u with n tokens of which the last c are candidates (h = n - c),
+ *   local token indices i, j in [0, n):
+ *     position      p(i)   = min(i, h)
+ *     allowed       M(i,j) = j <= i                 for history rows (i < h)
+ *                            j < h  or  j == i      for candidate rows (i >= h)
+ *     time bucket   b(i,j) = clamp(floor(ln(|t_i - t_j| + 1) / 0.301), 0, NB - 1)
+ *     score         s(i,j) = alpha * <q_i, k_j> + rab_pos[p(i) - p(j) + n_max - 1]
+ *                            + rab_ts[b(i,j)]
+ *     weight        a(i,j) = SiLU(s(i,j)) / n_max on M(i,j), 0 elsewhere
+ *     per head      o_i    = sum_j a(i,j) v_j
+ *     output        y_i    = (LayerNorm(o_i) * gamma + beta) * u_i
+ *                            (LayerNorm over the H*d concatenated head features,
+ *                             biased variance, epsilon ln_eps)
+ *
+ * Sources (web pages on HSTU generative recommenders):
+ *   "Generative Recommenders at Scale" - Inside NVIDIA's GPU-native stack, and FAQ:
+ *       HSTU swaps softmax attention for SiLU weighting, a relative attention
+ *       bias and elementwise gating.
+ *   "How Generative Recommenders Are Redefining RecSys at Scale" - Summary and
+ *       Takeaways: timestamp-ordered interleaved items/actions; gating is
+ *       applied before the output projection.
+ *   "HSTU Generative Recommenders: Deploy on GPU Cloud" - M-FALCON section:
+ *       candidates scored in one pass with mask and relative bias modified so
+ *       that they share the history computation.
+ *   "Recomendador generativo HSTU com Dynamo-Triton" - KV cache section: the
+ *       cache keeps attention state of a stable prefix in a paged GPU table so
+ *       that only new actions and candidates are computed.
+ *
+ * Conventions
+ *   - The caller owns every buffer.  The library never allocates device or
+ *     host memory; scratch space is the caller's `workspace`.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  The return value covers host-side argument checks and
+ *     launch errors only.  Errors the device detects (bad offsets, lengths
+ *     above n_max, unsorted timestamps, page ids out of range, a wait that ran
+ *     out) are written to a status word inside the workspace and read with
+ *     hstu_check_device_error().
+ *   - Device pointers must be 16-byte aligned; q/k/v/u row strides must be
+ *     multiples of 8 elements (bf16) or 4 elements (fp32).
+ *   - `out` must not alias any input.
+ *   - Within one user, timestamps must be non-decreasing (the pages' inputs
+ *     are timestamp-ordered); the device reports HSTU_ERR_UNSORTED otherwise.
+ *   - No state is kept between calls; calls on different streams with
+ *     different workspaces may run concurrently.
+ */
+#ifndef HSTU_H_
+#define HSTU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#ifndef HSTU_STREAM_T_DEFINED
+#define HSTU_STREAM_T_DEFINED
+typedef struct CUstream_st* hstu_stream_t; /* same object as cudaStream_t */
+#endif
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARG = -1,   /* a NULL pointer, a non-positive size, an unknown flag      */
+  HSTU_ERR_UNSUPPORTED = -2,   /* a shape this build does not implement                     */
+  HSTU_ERR_ALIGNMENT = -3,     /* a pointer or stride breaks the 16-byte rule               */
+  HSTU_ERR_LENGTH = -4,        /* device: offsets not monotone, n > n_max, c > n, T mismatch */
+  HSTU_ERR_WORKSPACE = -5,     /* workspace too small                                        */
+  HSTU_ERR_CUDA = -6,          /* a CUDA runtime/driver call failed                          */
+  HSTU_ERR_TIMEOUT = -7,       /* device: a bounded wait inside a kernel ran out             */
+  HSTU_ERR_UNSORTED = -8,      /* device: timestamps decrease inside a user                  */
+  HSTU_ERR_PAGE = -9           /* device: a page-table entry outside [0, num_pages)          */
+} hstu_status;
+
+typedef enum { HSTU_DT_F32 = 0, HSTU_DT_BF16 = 1 } hstu_dtype;
+
+/* flags */
+#define HSTU_F_FORCE_SIMT     0x1u  /* use the CUDA-core kernel even where the tensor-core one applies */
+#define HSTU_F_OUTPUT_RAW_AV  0x2u  /* write o = A.V as fp32 [T,H,d] to `out` instead of y            */
+#define HSTU_F_STAGE_PLAN     0x10u /* run only the validate + tile-schedule kernels                    */
+#define HSTU_F_STAGE_ATTN     0x20u /* run only the attention kernel (needs a plan in the workspace)    */
+#define HSTU_F_STAGE_EPILOGUE 0x40u /* run only the LayerNorm-gate epilogue (needs the attention part)  */
+/* With none of the HSTU_F_STAGE_* bits set a call runs all three stages.  The
+ * split lets a caller time each kernel with events on its own stream; the
+ * stages must run in order on one stream with one workspace. */
+
+typedef struct {
+  int32_t batch;           /* B users                                                        */
+  int32_t num_heads;       /* H                                                              */
+  int32_t head_dim;        /* d = d_qk = d_v; tensor-core path: 128 (bf16); CUDA-core: 1..256 */
+  int32_t n_max;           /* N_max: rab_pos has 2*n_max-1 entries; every n <= n_max         */
+  int32_t num_ts_buckets;  /* NB entries of rab_ts, 1..128                                   */
+  int32_t total_tokens;    /* T: query rows (all tokens, or new tokens in paged mode)        */
+  int32_t max_seq_len;     /* host upper bound of n over users (paged: cached + new)          */
+  int32_t qkv_stride;      /* elements between consecutive tokens in q, k, v; 0 = H*d       */
+  int32_t u_stride;        /* elements between consecutive tokens in u; 0 = H*d             */
+  float alpha;             /* score scale, usually 1/sqrt(d)                                 */
+  float ln_eps;            /* LayerNorm epsilon, usually 1e-5                                */
+  hstu_dtype dtype;        /* type of q, k, v, u, the pool and out (raw-AV output is fp32)   */
+  uint32_t flags;          /* HSTU_F_*                                                       */
+} hstu_attn_params;
+
+/* Bytes of workspace hstu_attn_fwd needs for these parameters. */
+size_t hstu_attn_workspace_size(const hstu_attn_params* p);
+
+/*
+ * Jagged full-sequence forward (prefill / training-style forward, M-FALCON
+ * ranking when num_candidates is given).
+ *   q, k, v        [T, H, d] dtype, token stride qkv_stride
+ *   u              [T, H*d]  dtype, token stride u_stride
+ *   seq_offsets    [B+1] int32, seq_offsets[0] = 0, seq_offsets[B] = T
+ *   timestamps     [T] int64 seconds, non-decreasing inside each user
+ *   num_candidates [B] int32 or NULL (no candidates); the last c tokens of a
+ *                  user are its candidates
+ *   rab_pos        [2*n_max-1] fp32;  rab_ts [num_ts_buckets] fp32
+ *   ln_gamma, ln_beta  [H*d] fp32 or NULL (= 1 and = 0)
+ *   out            [T, H*d] dtype (fp32 [T,H,d] o with HSTU_F_OUTPUT_RAW_AV)
+ *   workspace      device scratch of at least hstu_attn_workspace_size() bytes
+ * Returns HSTU_OK or a negative hstu_status.
+ */
+int hstu_attn_fwd(const hstu_attn_params* p, const void* q, const void* k, const void* v,
+                  const void* u, const int32_t* seq_offsets, const int64_t* timestamps,
+                  const int32_t* num_candidates, const float* rab_pos, const float* rab_ts,
+                  const float* ln_gamma, const float* ln_beta, void* out, void* workspace,
+                  size_t workspace_bytes, hstu_stream_t stream);
+
+/* Bytes of workspace hstu_attn_fwd_paged needs with `num_splits` key splits. */
+size_t hstu_attn_paged_workspace_size(const hstu_attn_params* p, int32_t num_splits);
+
+/* A split count that fills the GPU for this problem (1..64). */
+int32_t hstu_attn_paged_default_splits(const hstu_attn_params* p, int32_t max_cached_len);
+
+/*
+ * Incremental forward over a paged K/V cache.  User u has cached_lens[u]
+ * prefix tokens whose K/V sit in the pools, plus new tokens given densely.
+ * The result for every new token equals the full-recompute result over
+ * prefix + new tokens (positions and timestamps count the prefix).
+ *   q_new, k_new, v_new [T_new, H, d]; u_new [T_new, H*d]   (T_new = p->total_tokens)
+ *   new_offsets   [B+1] int32 over the new tokens
+ *   timestamps    int64, per user cached_lens[u] + new tokens (prefix first),
+ *                 jagged by ts_offsets [B+1]
+ *   num_candidates [B] int32 or NULL: the last new tokens of a user are candidates
+ *   k_pool, v_pool [num_pages, H, page_size, d] dtype; slot s of page g holds
+ *                 token g_index*page_size + s of the user that owns the page
+ *   kv_page_table [B, max_pages_per_user] int32 physical page ids; entry
+ *                 (u, x) for x < ceil(cached_lens[u]/page_size) must be in
+ *                 [0, num_pages); other entries are not read
+ *   page_size     32, 64 or 128 (tensor-core path); any positive value (CUDA-core path)
+ *   num_splits    key splits per (user, head, query tile), 1..64
+ *   out           [T_new, H*d] dtype
+ */
+int hstu_attn_fwd_paged(const hstu_attn_params* p, const void* q_new, const void* k_new,
+                        const void* v_new, const void* u_new, const int32_t* new_offsets,
+                        const int64_t* timestamps, const int32_t* ts_offsets,
+                        const int32_t* num_candidates, const float* rab_pos,
+                        const float* rab_ts, const float* ln_gamma, const float* ln_beta,
+                        const void* k_pool, const void* v_pool, int32_t num_pages,
+                        const int32_t* kv_page_table, int32_t max_pages_per_user,
+                        int32_t page_size, const int32_t* cached_lens, int32_t num_splits,
+                        void* out, void* workspace, size_t workspace_bytes,
+                        hstu_stream_t stream);
+
+/*
+ * Time buckets of n time differences: out[i] = clamp(floor(ln(|dt[i]|+1)/0.301),
+ * 0, num_buckets-1), bit-exact for every int64 input.
+ *   dt [n] int64 device; out [n] int32 device; num_buckets 1..128.
+ */
+int hstu_ts_bucket(const int64_t* dt, int64_t n, int32_t num_buckets, int32_t* out,
+                   hstu_stream_t stream);
+
+/* Synchronises `stream`, then returns the status word the device wrote into
+ * `workspace` during the last call that used it (HSTU_OK if none). */
+int hstu_check_device_error(const void* workspace, hstu_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* hstu_status_string(int status);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int hstu_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_H_ */

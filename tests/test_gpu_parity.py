@@ -1,0 +1,331 @@
+"""GPU parity: the CUDA library through its C ABI against the fp64 oracle.
+
+Bar: bucket indices bit-exact; max-abs-err / max|Y| <= 1e-5 for fp32 inputs
+and <= 2e-2 for bf16 inputs.  Small cases compare every element; the full
+workload sizes compare sampled rows the oracle evaluates one by one, in the
+same launch configuration the bench times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import generative_recommender_attention_jagged_b200 as hstu
+import oracle
+import synth
+from tests import exact_bucket as eb
+from tests.gpu_helpers import (BF16_TOL, F32_TOL, dev, host64, rel_err, run_jagged, run_paged,
+                               sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from generative_recommender_attention_jagged_b200 import build
+    build.build()
+
+
+def small_batch(lengths, *, cands=None, H=4, d=128, n_max=None, seed=0, dtype=torch.bfloat16, scale=1.0):
+    rng = np.random.default_rng(seed)
+    n_max = n_max or max(8, int(max(lengths)))
+    return synth.jagged_batch(lengths, H, d, n_max, rng=rng, dtype=dtype, num_candidates=cands,
+                              qkvu_scale=scale)
+
+
+# ----------------------------------------------------------------------------
+# time buckets
+# ----------------------------------------------------------------------------
+
+def test_bucket_kernel_bit_exact_at_thresholds():
+    thr = eb.integer_thresholds()
+    xs = sorted({max(1, t + dl) for t in thr for dl in range(-2, 3) if t + dl - 1 < 2**63})
+    dts = np.array([x - 1 for x in xs] + [-(x - 1) for x in xs] + [2**63 - 1, -(2**63)], dtype=np.int64)
+    got = hstu.hstu_ts_bucket(dev(dts)).cpu().numpy()
+    want = np.array([eb.bucket(int(x)) for x in dts])
+    np.testing.assert_array_equal(got, want)
+
+
+def test_bucket_kernel_matches_oracle_random():
+    rng = np.random.default_rng(3)
+    n = (1 << 20) + 17  # ragged tail
+    dts = np.exp(rng.uniform(0, math.log(2.0**62), size=n)).astype(np.int64)
+    dts[::3] *= -1
+    got = hstu.hstu_ts_bucket(dev(dts)).cpu().numpy()
+    np.testing.assert_array_equal(got, oracle.ts_bucket(dts))
+
+
+@pytest.mark.parametrize("nb", [1, 16, 128])
+def test_bucket_kernel_clamps_to_table(nb):
+    dts = np.array([0, 5, 10**6, 10**15], dtype=np.int64)
+    got = hstu.hstu_ts_bucket(dev(dts), num_buckets=nb).cpu().numpy()
+    np.testing.assert_array_equal(got, oracle.ts_bucket(dts, nb))
+
+
+def test_bucket_kernel_empty():
+    out = hstu.hstu_ts_bucket(torch.zeros(0, dtype=torch.int64, device="cuda"))
+    assert out.numel() == 0
+
+
+# ----------------------------------------------------------------------------
+# fp32 (CUDA-core kernel)
+# ----------------------------------------------------------------------------
+
+def test_tiny_fp32_workload_full():
+    b = synth.workload_attention("tiny_fp32")
+    y = host64(run_jagged(b))
+    assert rel_err(y, oracle.batch_attn(b)) <= F32_TOL
+
+
+def test_tiny_fp32_raw_av_and_candidates():
+    b = small_batch([37, 64, 1, 20], cands=[5, 0, 1, 20], H=2, d=32, n_max=64, dtype=torch.float32,
+                    scale=1 / math.sqrt(32))
+    rng = np.random.default_rng(9)
+    b.ln_gamma = rng.normal(size=64).astype(np.float32)
+    b.ln_beta = rng.normal(size=64).astype(np.float32)
+    y = host64(run_jagged(b))
+    want_y, want_o = oracle.batch_attn(b, want_o=True)
+    assert rel_err(y, want_y) <= F32_TOL
+    o = host64(run_jagged(b, raw_av=True))
+    assert rel_err(o, want_o) <= F32_TOL
+
+
+@pytest.mark.parametrize("d", [1, 8, 33, 64, 200])
+def test_fp32_odd_head_dims(d):
+    b = small_batch([9, 17, 3], cands=[0, 4, 0], H=3, d=d, n_max=20, dtype=torch.float32, seed=d)
+    if (3 * d) % 4:
+        pytest.skip("fp32 row stride must be a multiple of 4 elements")
+    assert rel_err(host64(run_jagged(b)), oracle.batch_attn(b)) <= F32_TOL
+
+
+# ----------------------------------------------------------------------------
+# bf16 tensor-core kernel, small shapes: every element
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lengths,cands", [
+    ([128], None),                         # one exact tile
+    ([1, 2, 127, 129, 300], None),         # ragged tails, tiny users
+    ([513, 200, 64], [0, 0, 0]),           # several tiles, candidates given but zero
+    ([700, 300], [100, 300]),              # candidates; a user made only of candidates
+    ([260, 140, 257], [130, 7, 129]),      # candidate block across tile edges
+])
+def test_bf16_tensor_core_small(lengths, cands):
+    b = small_batch(lengths, cands=cands, n_max=max(lengths) + 64, seed=len(lengths))
+    want_y, want_o = oracle.batch_attn(b, want_o=True)
+    o = host64(run_jagged(b, raw_av=True))
+    assert rel_err(o, want_o) <= BF16_TOL
+    y = host64(run_jagged(b))
+    assert rel_err(y, want_y) <= BF16_TOL
+
+
+def test_bf16_tensor_core_matches_cuda_core_kernel():
+    b = small_batch([400, 131, 77], cands=[50, 0, 3], n_max=512, seed=5)
+    o_tc = host64(run_jagged(b, raw_av=True))
+    o_simt = host64(run_jagged(b, raw_av=True, force_simt=True))
+    assert rel_err(o_tc, o_simt) <= BF16_TOL
+    _, want_o = oracle.batch_attn(b, want_o=True)
+    assert rel_err(o_simt, want_o) <= 1e-4  # fp32 math on bf16 inputs
+
+
+def test_bf16_gamma_beta_and_strided_views():
+    # q/k/v/u as column blocks of one [T, 4*H*d] buffer, as the layer's f1 output is laid out
+    b = small_batch([300, 45], cands=[20, 0], n_max=400, seed=11)
+    rng = np.random.default_rng(1)
+    b.ln_gamma = rng.normal(size=512).astype(np.float32)
+    b.ln_beta = rng.normal(size=512).astype(np.float32)
+    T = b.total_tokens
+    big = torch.cat([b.u.view(T, 512), b.v.view(T, 512), b.q.view(T, 512), b.k.view(T, 512)], 1).cuda()
+    u, v, q, k = (big[:, i * 512:(i + 1) * 512] for i in range(4))
+    out = hstu.hstu_attn_fwd(q.view(T, 4, 128), k.view(T, 4, 128), v.view(T, 4, 128), u,
+                             dev(b.seq_offsets, torch.int32), dev(b.timestamps, torch.int64),
+                             dev(b.rab_pos, torch.float32), dev(b.rab_ts, torch.float32), n_max=b.n_max,
+                             num_candidates=dev(b.num_candidates, torch.int32),
+                             ln_gamma=dev(b.ln_gamma), ln_beta=dev(b.ln_beta))
+    torch.cuda.synchronize()
+    assert rel_err(host64(out), oracle.batch_attn(b)) <= BF16_TOL
+
+
+def test_bf16_larger_bias_magnitudes():
+    # biases of order 1 exercise the bucket walk and position window far from zero
+    b = small_batch([1000, 333], cands=[0, 33], n_max=1400, seed=21)
+    rng = np.random.default_rng(2)
+    b.rab_pos = rng.normal(0, 1.0, size=2 * b.n_max - 1).astype(np.float32)
+    b.rab_ts = rng.normal(0, 1.0, size=128).astype(np.float32)
+    _, want_o = oracle.batch_attn(b, want_o=True)
+    assert rel_err(host64(run_jagged(b, raw_av=True)), want_o) <= BF16_TOL
+
+
+def test_one_hot_time_bias_selects_exact_buckets():
+    # with q = k = 0 and rab_pos = 0, only keys in the one-hot bucket contribute:
+    # any bucket error on the GPU shows up as a whole missing/extra v row
+    b = small_batch([600, 250], n_max=700, seed=4)
+    b.q.zero_()
+    b.k.zero_()
+    b.rab_pos[:] = 0
+    for bstar in (19, 23, 30):
+        b.rab_ts[:] = 0
+        b.rab_ts[bstar] = 4.0
+        _, want_o = oracle.batch_attn(b, want_o=True)
+        got = host64(run_jagged(b, raw_av=True))
+        assert rel_err(got, want_o) <= 1e-2, bstar
+
+
+# ----------------------------------------------------------------------------
+# invariants on the GPU
+# ----------------------------------------------------------------------------
+
+def test_gpu_causality_bitwise():
+    b = small_batch([520], n_max=600, seed=7)
+    y0 = run_jagged(b).cpu()
+    i0 = 300
+    for t in (b.q, b.k, b.v, b.u):
+        t[i0 + 1:] = torch.randn_like(t[i0 + 1:].float()).to(t.dtype)
+    y1 = run_jagged(b).cpu()
+    assert torch.equal(y0[:i0 + 1], y1[:i0 + 1])
+    assert not torch.equal(y0[i0 + 1:], y1[i0 + 1:])
+
+
+def test_gpu_jagged_batch_equals_per_user_runs():
+    b = small_batch([300, 129, 1, 450], cands=[0, 9, 0, 60], n_max=500, seed=8)
+    y = run_jagged(b).cpu()
+    off = b.seq_offsets
+    for u in range(b.batch):
+        lo, hi = int(off[u]), int(off[u + 1])
+        bu = synth.JaggedBatch(q=b.q[lo:hi], k=b.k[lo:hi], v=b.v[lo:hi], u=b.u[lo:hi],
+                               seq_offsets=np.array([0, hi - lo], np.int32), timestamps=b.timestamps[lo:hi],
+                               num_candidates=b.num_candidates[u:u + 1], rab_pos=b.rab_pos, rab_ts=b.rab_ts,
+                               alpha=b.alpha, n_max=b.n_max, num_heads=b.num_heads, head_dim=b.head_dim)
+        assert torch.equal(run_jagged(bu).cpu(), y[lo:hi]), u
+
+
+def test_gpu_candidate_permutation_equivariance():
+    n, c = 400, 150
+    b = small_batch([n], cands=[c], n_max=512, seed=10)
+    y0 = host64(run_jagged(b))
+    h = n - c
+    perm = np.array(list(range(h)) + list(h + np.random.default_rng(0).permutation(c)))
+    for name in ("q", "k", "v", "u"):
+        setattr(b, name, getattr(b, name)[perm].clone())
+    b.timestamps = b.timestamps[perm]
+    y1 = host64(run_jagged(b))
+    assert rel_err(y1, y0[perm]) <= 1e-6
+
+
+# ----------------------------------------------------------------------------
+# device-detected errors (the kernels' own checks; nothing out of bounds is read)
+# ----------------------------------------------------------------------------
+
+def _status(b, **kw):
+    ws = torch.empty(hstu.hstu_attn_workspace_size(hstu.attn_params(
+        batch=b.batch, num_heads=b.num_heads, head_dim=b.head_dim, n_max=b.n_max, total_tokens=b.total_tokens,
+        max_seq_len=b.n_max, dtype=b.q.dtype)), dtype=torch.uint8, device="cuda")
+    run_jagged(b, workspace=ws, **kw)
+    return hstu.hstu_check_device_error(ws)
+
+
+def test_device_reports_unsorted_timestamps():
+    b = small_batch([200, 100], n_max=256)
+    assert _status(b) == 0
+    b.timestamps = b.timestamps.copy()
+    b.timestamps[250] = b.timestamps[249] - 5
+    assert _status(b) == -8
+
+
+def test_device_reports_length_above_n_max():
+    b = small_batch([200, 100], n_max=256)
+    b.n_max = 150
+    b.rab_pos = b.rab_pos[:2 * 150 - 1]
+    assert _status(b) == -4
+
+
+def test_device_reports_too_many_candidates():
+    b = small_batch([200, 100], cands=[0, 5], n_max=256)
+    b.num_candidates = np.array([0, 101], np.int32)
+    assert _status(b) == -4
+
+
+# ----------------------------------------------------------------------------
+# paged incremental mode
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cached,acts,cands,page,splits", [
+    ([300, 128, 0, 77], [5, 64, 3, 1], [2, 64, 0, 1], 32, 1),
+    ([1000, 520], [64, 1], [64, 0], 32, 3),
+    ([256, 130], [10, 20], [4, 0], 64, 2),
+    ([511, 129], [100, 140], [28, 0], 128, 4),
+])
+def test_paged_small_matches_oracle(cached, acts, cands, page, splits):
+    rng = np.random.default_rng(sum(cached))
+    n_max = max(c + a + k for c, a, k in zip(cached, acts, cands)) + 16
+    pb = synth.paged_batch(cached, acts, cands, 4, 128, n_max, rng=rng, page_size=page)
+    want_y, want_o = oracle.batch_paged(pb, want_o=True)
+    o = host64(run_paged(pb, raw_av=True, num_splits=splits))
+    assert np.isfinite(o).all()  # the NaN-poisoned pool slots are never read into the result
+    assert rel_err(o, want_o) <= BF16_TOL
+    y = host64(run_paged(pb, num_splits=splits))
+    assert rel_err(y, want_y) <= BF16_TOL
+
+
+def test_paged_cuda_core_kernel_matches_oracle():
+    rng = np.random.default_rng(5)
+    pb = synth.paged_batch([100, 37], [6, 3], [2, 1], 2, 64, 160, rng=rng, page_size=16, dtype=torch.float32)
+    assert rel_err(host64(run_paged(pb, force_simt=True)), oracle.batch_paged(pb)) <= F32_TOL
+
+
+def test_paged_equals_full_recompute_on_gpu():
+    rng = np.random.default_rng(6)
+    pb = synth.paged_batch([700, 333], [64, 10], [64, 5], 4, 128, 900, rng=rng)
+    y_paged = host64(run_paged(pb, num_splits=2))
+    qs, ks, vs, us, lens = [], [], [], [], []
+    for u in range(pb.batch):
+        lo, hi = pb.new_offsets[u], pb.new_offsets[u + 1]
+        L = int(pb.cached_lens[u])
+        qs += [torch.zeros(L, 4, 128, dtype=torch.bfloat16), pb.q[lo:hi]]
+        ks += [pb.k_prefix[u], pb.k[lo:hi]]
+        vs += [pb.v_prefix[u], pb.v[lo:hi]]
+        us += [torch.zeros(L, 512, dtype=torch.bfloat16), pb.u[lo:hi]]
+        lens.append(L + hi - lo)
+    full = synth.JaggedBatch(q=torch.cat(qs), k=torch.cat(ks), v=torch.cat(vs), u=torch.cat(us),
+                             seq_offsets=synth.offsets_from_lengths(lens), timestamps=pb.timestamps,
+                             num_candidates=pb.num_candidates, rab_pos=pb.rab_pos, rab_ts=pb.rab_ts,
+                             alpha=pb.alpha, n_max=pb.n_max, num_heads=4, head_dim=128)
+    y_full = host64(run_jagged(full))
+    rows = np.concatenate([np.arange(full.seq_offsets[u] + pb.cached_lens[u], full.seq_offsets[u + 1])
+                           for u in range(pb.batch)])
+    assert rel_err(y_paged, y_full[rows]) <= BF16_TOL
+
+
+def test_device_reports_bad_page_id():
+    rng = np.random.default_rng(7)
+    pb = synth.paged_batch([100, 64], [4, 4], [1, 1], 4, 128, 200, rng=rng)
+    pb.kv_page_table = pb.kv_page_table.copy()
+    pb.kv_page_table[1, 0] = pb.k_pool.shape[0] + 3
+    params = hstu.attn_params(batch=2, num_heads=4, head_dim=128, n_max=200, total_tokens=int(pb.new_offsets[-1]),
+                              max_seq_len=200, dtype=torch.bfloat16)
+    ws = torch.empty(hstu.hstu_attn_paged_workspace_size(params, 2), dtype=torch.uint8, device="cuda")
+    run_paged(pb, num_splits=2, workspace=ws)
+    assert hstu.hstu_check_device_error(ws) == -9
+
+
+# ----------------------------------------------------------------------------
+# full workload sizes: sampled rows, the bench's launch configuration
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["layer_bf16", "stack8_bf16", "mfalcon_bf16"])
+def test_workload_sampled_rows(name):
+    b = synth.workload_attention(name, layer=0)
+    y = host64(run_jagged(b))
+    assert np.isfinite(y).all()
+    rows = sample_rows(b.seq_offsets, b.num_candidates, per_user=4)
+    want = oracle.batch_attn(b, rows=rows)
+    assert rel_err(y[rows], want) <= BF16_TOL
+
+
+def test_paged_workload_sampled_rows():
+    pb = synth.workload_paged(layer=0)
+    y = host64(run_paged(pb))
+    assert np.isfinite(y).all()
+    rows = sample_rows(pb.new_offsets, pb.num_candidates, per_user=6)
+    want = oracle.batch_paged(pb, rows=rows)
+    assert rel_err(y[rows], want) <= BF16_TOL

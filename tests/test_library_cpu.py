@@ -1,0 +1,117 @@
+"""CPU-only checks of the C ABI: the library builds, loads, exports every
+symbol include/hstu.h declares, and rejects bad host arguments before it
+touches a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import generative_recommender_attention_jagged_b200 as hstu
+from generative_recommender_attention_jagged_b200 import _lib, build as hbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hstu.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s*(hstu_[a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hbuild.build()
+    return _lib.load()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("hstu_attn_fwd", "hstu_attn_fwd_paged", "hstu_ts_bucket", "hstu_attn_workspace_size",
+                     "hstu_check_device_error", "hstu_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_params_struct_matches_header(lib):
+    assert ctypes.sizeof(_lib.AttnParams) == 13 * 4
+
+
+def test_status_strings(lib):
+    assert hstu.hstu_status_string(0) == "HSTU_OK"
+    for code in range(-9, 0):
+        assert hstu.hstu_status_string(code).startswith(_lib.STATUS_NAMES[code])
+    assert hstu.hstu_version() == 100
+
+
+def params(**kw):
+    base = dict(batch=2, num_heads=4, head_dim=128, n_max=1024, total_tokens=300, max_seq_len=200,
+                dtype=__import__("torch").bfloat16)
+    base.update(kw)
+    return hstu.attn_params(**base)
+
+
+def test_workspace_size_grows_with_tokens_and_splits(lib):
+    small = hstu.hstu_attn_workspace_size(params())
+    big = hstu.hstu_attn_workspace_size(params(total_tokens=3000))
+    assert 0 < small < big
+    assert small >= 256 + 300 * 512 * 4
+    assert hstu.hstu_attn_paged_workspace_size(params(), 4) >= hstu.hstu_attn_paged_workspace_size(params(), 1)
+
+
+@pytest.mark.parametrize("bad", [dict(batch=0), dict(num_heads=0), dict(n_max=0), dict(num_ts_buckets=129),
+                                 dict(head_dim=300), dict(flags=0x1000)])
+def test_bad_params_rejected_on_host(lib, bad):
+    p = params(**bad)
+    assert lib.hstu_attn_workspace_size(ctypes.byref(p)) == 0
+    rc = lib.hstu_attn_fwd(ctypes.byref(p), *([None] * 13), 0, None)
+    assert rc in (-1, -2)
+
+
+def test_null_pointers_rejected_on_host(lib):
+    p = params()
+    rc = lib.hstu_attn_fwd(ctypes.byref(p), *([None] * 13), 0, None)
+    assert rc == -1
+    rc = lib.hstu_attn_fwd_paged(ctypes.byref(p), *([None] * 14), 1, None, 1, 32, None, 1, None, None, 0, None)
+    assert rc == -1
+
+
+def test_misaligned_pointer_rejected_on_host(lib):
+    p = params()
+    fake = [ctypes.c_void_p(0x1000)] * 13
+    fake[0] = ctypes.c_void_p(0x1008)  # q not 16-byte aligned
+    rc = lib.hstu_attn_fwd(ctypes.byref(p), *fake, 1 << 30, None)
+    assert rc == -3
+
+
+def test_small_workspace_rejected_on_host(lib):
+    p = params(flags=_lib.F_FORCE_SIMT)
+    fake = [ctypes.c_void_p(0x1000)] * 13
+    rc = lib.hstu_attn_fwd(ctypes.byref(p), *fake, 64, None)
+    assert rc == -5
+
+
+def test_bucket_kernel_rejects_bad_args_on_host(lib):
+    assert lib.hstu_ts_bucket(None, -1, 128, None, None) == -1
+    assert lib.hstu_ts_bucket(None, 10, 128, None, None) == -1
+    assert lib.hstu_ts_bucket(None, 0, 0, None, None) == -1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(4, 1, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        hstu.hstu_attn_fwd(q, q, q, q.view(4, 128), torch.tensor([0, 4], dtype=torch.int32),
+                           torch.zeros(4, dtype=torch.int64), torch.zeros(7), torch.zeros(128), n_max=4)
