@@ -106,9 +106,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
+  const WorkItem it = a.items[item_idx];
+  // a work list not written by this call's scheduler must not send us out of bounds
+  if (it.user < 0 || it.user >= a.B || it.head < 0 || it.head >= a.H || it.split < 0 ||
+      it.split >= a.num_splits || it.qtile < 0 ||
+      it.qtile * kTile >= a.q_offsets[it.user + 1] - a.q_offsets[it.user])
+    return;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const WorkItem it = a.items[item_idx];
   const TileGeom g = tile_geom(a, it.user, it.qtile);
   int tb, te;
   split_range(g.n_tiles, it.split, a.num_splits, tb, te);

@@ -154,7 +154,8 @@ int run(const hstu_attn_params* p, const Common& c) {
   for (const void* ptr : ptrs)
     if (ptr && !aligned16(ptr)) return HSTU_ERR_ALIGNMENT;
   const bool tc = use_tensor_cores(p);
-  if (tc && c.paged && (c.page_size > kTile || kTile % c.page_size)) return HSTU_ERR_UNSUPPORTED;
+  // tensor-core path: whole pages land as 1024-byte-aligned swizzled boxes
+  if (tc && c.paged && (c.page_size < 8 || c.page_size > kTile || kTile % c.page_size)) return HSTU_ERR_UNSUPPORTED;
   const Layout l = layout_for(p, tc ? c.splits : 1, tc);
   if (c.ws_bytes < l.total) return HSTU_ERR_WORKSPACE;
 

@@ -150,7 +150,7 @@ int32_t hstu_attn_paged_default_splits(const hstu_attn_params* p, int32_t max_ca
  *   kv_page_table [B, max_pages_per_user] int32 physical page ids; entry
  *                 (u, x) for x < ceil(cached_lens[u]/page_size) must be in
  *                 [0, num_pages); other entries are not read
- *   page_size     32, 64 or 128 (tensor-core path); any positive value (CUDA-core path)
+ *   page_size     8, 16, 32, 64 or 128 (tensor-core path); any positive value (CUDA-core path)
  *   num_splits    key splits per (user, head, query tile), 1..64
  *   out           [T_new, H*d] dtype
  */

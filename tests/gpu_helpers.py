@@ -22,7 +22,6 @@ def dev(x, dtype=None):
 
 
 def run_jagged(b, *, raw_av=False, force_simt=False, workspace=None, check_status=True, **kw):
-    ws_out = {}
     out = hstu.hstu_attn_fwd(dev(b.q), dev(b.k), dev(b.v), dev(b.u), dev(b.seq_offsets, torch.int32),
                              dev(b.timestamps, torch.int64), dev(b.rab_pos, torch.float32),
                              dev(b.rab_ts, torch.float32), n_max=b.n_max, alpha=b.alpha,

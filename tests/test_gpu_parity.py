@@ -329,3 +329,13 @@ def test_paged_workload_sampled_rows():
     rows = sample_rows(pb.new_offsets, pb.num_candidates, per_user=6)
     want = oracle.batch_paged(pb, rows=rows)
     assert rel_err(y[rows], want) <= BF16_TOL
+
+
+def test_tensor_core_path_is_the_one_that_runs():
+    # the two kernels round differently (bf16 P and tanh.approx vs fp32 expf), so
+    # bitwise-different outputs show the bf16 d=128 call did not take the CUDA-core kernel
+    b = small_batch([300], n_max=320, seed=12)
+    o_tc = run_jagged(b, raw_av=True).cpu()
+    o_simt = run_jagged(b, raw_av=True, force_simt=True).cpu()
+    assert not torch.equal(o_tc, o_simt)
+    assert rel_err(host64(o_tc), host64(o_simt)) <= BF16_TOL
