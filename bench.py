@@ -1,0 +1,493 @@
+"""HSTU jagged attention forward benchmark on B200.
+
+Workload (default): the 8-layer HSTU stack workload at sequence lengths up to
+8,320 -- 8 users with lengths uniform in [4160, 8320], 4 heads, d = 128,
+N_max = 8320, causal mask, per-layer rab tables and Q/K/V/U, bf16 inputs.
+One step = the attention forward (validate + tile schedule, tcgen05 attention,
+LayerNorm-gate epilogue) of all 8 layers.  The metric is attention TFLOP/s
+(algorithmic: 2 (d_qk + d_v) flops per allowed (query, key) pair and head),
+with tokens/s alongside.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); users are independent, so every
+rank runs its own batch with no collective on the data path (weak scaling);
+timing is the max over ranks.  --impl reference times the fp64 CPU oracle on
+the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+FLOPS_PER_PAIR_HEAD = 2 * (128 + 128)  # QK^T and AV, d_qk = d_v = 128
+TILE = 128
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention-kernel launch
+# (per layer of this workload), from the ncu capture summarised in
+# profiles/attn_sm100_stack8.md; None until a capture of the current kernel exists.
+ATTN_TRAFFIC_BYTES = None
+
+
+def allowed_pairs(lengths, cands=None):
+    """Allowed (query, key) pairs per head: h(h+1)/2 causal history pairs plus,
+    per candidate, the h history keys and itself."""
+    total = 0
+    for i, n in enumerate(lengths):
+        c = 0 if cands is None else int(cands[i])
+        h = int(n) - c
+        total += h * (h + 1) // 2 + c * (h + 1)
+    return total
+
+
+def issued_tiles(lengths, cands=None):
+    """128x128 key tiles the tensor-core kernel issues (both GEMMs), per head."""
+    tiles = 0
+    for i, n in enumerate(lengths):
+        c = 0 if cands is None else int(cands[i])
+        h = int(n) - c
+        for m in range(math.ceil(int(n) / TILE)):
+            q_last = min(int(n), (m + 1) * TILE) - 1
+            kv_end = max(0, min(q_last + 1, h))
+            tiles += math.ceil(kv_end / TILE)
+    return tiles
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(batch, target_s: float, seed: int = 0):
+    """Time the fp64 oracle on random query rows of `batch` for about target_s."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    lengths = batch.lengths
+    off = batch.seq_offsets
+    # inputs converted to fp64 once, outside the timed calls
+    q64, k64, v64, u64 = (t.double().numpy() for t in (batch.q, batch.k, batch.v, batch.u))
+    # per-row keys of a causal row i: i + 1
+    def run(nrows):
+        users = rng.integers(0, batch.batch, size=nrows)
+        rows = np.array([off[usr] + rng.integers(0, lengths[usr]) for usr in users], dtype=np.int64)
+        keys = 0
+        for r, usr in zip(rows, users):
+            i = r - off[usr]
+            c = 0 if batch.num_candidates is None else int(batch.num_candidates[usr])
+            h = lengths[usr] - c
+            keys += (i + 1) if i < h else (h + 1)
+        t0 = time.perf_counter()
+        oracle.attn_jagged(q64, k64, v64, u64, batch.seq_offsets, batch.timestamps, batch.num_candidates,
+                           batch.rab_pos, batch.rab_ts, batch.alpha, batch.n_max, rows=rows)
+        return time.perf_counter() - t0, keys * batch.num_heads * FLOPS_PER_PAIR_HEAD, nrows
+    dt, _, _ = run(8)  # warm-up
+    dt, flops, nrows = run(16)
+    n = int(max(16, min(20000, 16 * target_s / max(dt, 1e-3))))
+    dt, flops, nrows = run(n)
+    return dt, flops, nrows
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def to_dev(x, dtype=None, device="cuda"):
+    if x is None:
+        return None
+    if isinstance(x, np.ndarray):
+        x = torch.from_numpy(np.ascontiguousarray(x))
+    return x.to(device=device, dtype=dtype) if dtype is not None else x.to(device)
+
+
+def run_ours(args, rank, world, device):
+    import generative_recommender_attention_jagged_b200 as hstu
+    from generative_recommender_attention_jagged_b200 import _lib
+
+    seed = None if rank == 0 else 1000 + 7919 * rank  # every rank its own users
+    layers = synth.attention_stack(args.workload, num_layers=args.layers, seed=seed)
+    L = len(layers)
+    b0 = layers[0]
+    T, H, d = b0.q.shape
+    stream = torch.cuda.current_stream()
+    dev_layers = []
+    for b in layers:
+        dev_layers.append(dict(q=to_dev(b.q), k=to_dev(b.k), v=to_dev(b.v), u=to_dev(b.u),
+                               rab_pos=to_dev(b.rab_pos, torch.float32), rab_ts=to_dev(b.rab_ts, torch.float32)))
+    off = to_dev(b0.seq_offsets, torch.int32)
+    ts = to_dev(b0.timestamps, torch.int64)
+    cand = to_dev(b0.num_candidates, torch.int32)
+    params = hstu.attn_params(batch=b0.batch, num_heads=H, head_dim=d, n_max=b0.n_max, total_tokens=T,
+                              max_seq_len=b0.max_seq_len, dtype=b0.q.dtype, alpha=b0.alpha)
+    ws_bytes = hstu.hstu_attn_workspace_size(params)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    outs = [torch.empty(T, H * d, dtype=b0.q.dtype, device=device) for _ in range(L)]
+
+    def call(l, stage):
+        x = dev_layers[l]
+        return hstu.hstu_attn_fwd(x["q"], x["k"], x["v"], x["u"], off, ts, x["rab_pos"], x["rab_ts"],
+                                  n_max=b0.n_max, alpha=b0.alpha, num_candidates=cand,
+                                  max_seq_len=b0.max_seq_len, out=outs[l], workspace=ws, stages=stage)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps * L)]
+
+    def step(timed_idx=None):
+        for l in range(L):
+            call(l, _lib.F_STAGE_PLAN)
+            if timed_idx is not None:
+                ev[timed_idx * L + l][0].record(stream)
+            call(l, _lib.F_STAGE_ATTN)
+            if timed_idx is not None:
+                ev[timed_idx * L + l][1].record(stream)
+            call(l, _lib.F_STAGE_EPILOGUE)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = hstu.hstu_check_device_error(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} ({hstu.hstu_status_string(status)})")
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        step(s)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        tt = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+
+    lengths = b0.lengths
+    pairs = allowed_pairs(lengths, b0.num_candidates)
+    flops_layer = pairs * H * FLOPS_PER_PAIR_HEAD
+    flops_step = flops_layer * L
+    ms_step = total_ms / args.steps
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    tokens_s = T * L * world / (ms_step * 1e-3)
+    attn_avg_ms = float(np.mean(attn_ms))
+    achieved = flops_layer / (attn_avg_ms * 1e-3) / 1e12
+    tiles = issued_tiles(lengths, b0.num_candidates) * H
+    issued_tflops = tiles * 2 * (2 * TILE * TILE * 128) / (attn_avg_ms * 1e-3) / 1e12
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+
+    # ---- end to end through the C ABI from pinned host buffers ----
+    e2e = None
+    if args.e2e_steps > 0:
+        host = []
+        for b in layers:
+            host.append({k: (v.pin_memory() if isinstance(v, torch.Tensor) else torch.from_numpy(v).pin_memory())
+                         for k, v in dict(q=b.q, k=b.k, v=b.v, u=b.u, rab_pos=b.rab_pos, rab_ts=b.rab_ts).items()})
+        h_off = torch.from_numpy(b0.seq_offsets.astype(np.int32)).pin_memory()
+        h_ts = torch.from_numpy(b0.timestamps).pin_memory()
+        h_out = [torch.empty(T, H * d, dtype=b0.q.dtype).pin_memory() for _ in range(L)]
+        d_in = {k: torch.empty_like(v, device=device) for k, v in host[0].items()}
+        d_off = torch.empty_like(h_off, device=device)
+        d_ts = torch.empty_like(h_ts, device=device)
+        d_out = torch.empty(T, H * d, dtype=b0.q.dtype, device=device)
+        h2d = d2h = 0
+
+        def e2e_step(count):
+            nonlocal h2d, d2h
+            d_off.copy_(h_off, non_blocking=True)
+            d_ts.copy_(h_ts, non_blocking=True)
+            if count:
+                h2d += h_off.numel() * 4 + h_ts.numel() * 8
+            for l in range(L):
+                for k_, v_ in host[l].items():
+                    d_in[k_].copy_(v_, non_blocking=True)
+                    if count:
+                        h2d += v_.numel() * v_.element_size()
+                hstu.hstu_attn_fwd(d_in["q"], d_in["k"], d_in["v"], d_in["u"], d_off, d_ts, d_in["rab_pos"],
+                                   d_in["rab_ts"], n_max=b0.n_max, alpha=b0.alpha, max_seq_len=b0.max_seq_len,
+                                   out=d_out, workspace=ws)
+                h_out[l].copy_(d_out, non_blocking=True)
+                if count:
+                    d2h += d_out.numel() * d_out.element_size()
+
+        e2e_step(False)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step(True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=device, dtype=torch.float64)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e_step = e_ms / args.e2e_steps
+        e2e = {"value": round(flops_step * world / (e_step * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "ms_per_step": round(e_step, 3), "steps": args.e2e_steps,
+               "h2d_bytes_per_step": h2d // args.e2e_steps, "d2h_bytes_per_step": d2h // args.e2e_steps}
+
+    result = {
+        "metric": "HSTU attention fwd TFLOP/s + tokens/s, % of B200 BF16 peak / HBM BW",
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; no dataset)",
+        "config": {"workload": f"{args.workload}: 8-layer HSTU attention, B={b0.batch} users, lengths "
+                               f"U[4160,8320] (T={T}), H={H}, d={d}, N_max={b0.n_max}, causal",
+                   "global_batch": b0.batch * world, "total_tokens_per_gpu": T, "layers": L,
+                   "parallelism": f"replicas x{world} (users sharded, no collective)",
+                   "l2": "inputs larger than L2 (8 per-layer Q/K/V/U sets, %.2f GB)" %
+                         (4 * T * H * d * 2 * L / 1e9)},
+        "tokens_per_s": round(tokens_s, 1),
+        "roofline": {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "traffic": ATTN_TRAFFIC_BYTES,
+                     "launch_ms": round(attn_avg_ms, 4), "flops_per_launch": flops_layer,
+                     "issued_tile_tflops": round(issued_tflops, 2),
+                     "issued_frac": round(issued_tflops / peak, 4)},
+        "gpu_launches": args.steps * L * 4,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    return result, b0
+
+
+def run_paged_bench(args, device):
+    """Paged incremental workload: 8 users, cached prefix U[6144,8192] in
+    32-token pages, +64 actions +64 candidates, 8 layers with separate pools."""
+    import generative_recommender_attention_jagged_b200 as hstu
+    from generative_recommender_attention_jagged_b200 import _lib
+    layers = synth.paged_stack(8)
+    stream = torch.cuda.current_stream()
+    dl = []
+    for pb in layers:
+        dl.append(dict(q=to_dev(pb.q), k=to_dev(pb.k), v=to_dev(pb.v), u=to_dev(pb.u),
+                       off=to_dev(pb.new_offsets, torch.int32), ts=to_dev(pb.timestamps, torch.int64),
+                       tso=to_dev(pb.ts_offsets, torch.int32), cand=to_dev(pb.num_candidates, torch.int32),
+                       rp=to_dev(pb.rab_pos, torch.float32), rt=to_dev(pb.rab_ts, torch.float32),
+                       kp=to_dev(pb.k_pool), vp=to_dev(pb.v_pool), pt=to_dev(pb.kv_page_table, torch.int32),
+                       cl=to_dev(pb.cached_lens, torch.int32)))
+    pb0 = layers[0]
+    T = int(pb0.new_offsets[-1])
+    maxc = int(pb0.cached_lens.max())
+    params = hstu.attn_params(batch=pb0.batch, num_heads=4, head_dim=128, n_max=pb0.n_max, total_tokens=T,
+                              max_seq_len=pb0.n_max, dtype=torch.bfloat16)
+    splits = hstu.hstu_attn_paged_default_splits(params, maxc)
+    ws = torch.empty(hstu.hstu_attn_paged_workspace_size(params, splits), dtype=torch.uint8, device=device)
+    out = torch.empty(T, 512, dtype=torch.bfloat16, device=device)
+
+    def call(x, stage):
+        hstu.hstu_attn_fwd_paged(x["q"], x["k"], x["v"], x["u"], x["off"], x["ts"], x["tso"], x["rp"], x["rt"],
+                                 x["kp"], x["vp"], x["pt"], x["cl"], n_max=pb0.n_max, num_candidates=x["cand"],
+                                 num_splits=splits, out=out, workspace=ws, stages=stage)
+
+    steps = max(3, min(args.steps, 50))
+    for _ in range(3):
+        for x in dl:
+            call(x, 0)
+    torch.cuda.synchronize()
+    ev = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        for x in dl:
+            call(x, _lib.F_STAGE_PLAN)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call(x, _lib.F_STAGE_ATTN)
+            b.record(stream)
+            call(x, _lib.F_STAGE_EPILOGUE)
+            ev.append((a, b))
+    t1.record(stream)
+    torch.cuda.synchronize()
+    status = hstu.hstu_check_device_error(ws)
+    if status != 0:
+        raise RuntimeError(f"paged device status {status}")
+    ms_layer = t0.elapsed_time(t1) / (steps * len(dl))
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    kv_bytes = int(sum(2 * int(c) * 4 * 128 * 2 for c in pb0.cached_lens))
+    new_bytes = T * 512 * 2 * 4 + int(pb0.ts_offsets[-1]) * 8
+    alg_bytes = kv_bytes + new_bytes
+    peaks, kind = measured_peaks()
+    achieved = alg_bytes / (attn_ms * 1e-3) / 1e9
+    return {"workload": "paged_bf16: 8 users, cached U[6144,8192] in 32-token pages, +64 actions "
+                        "+64 candidates, 8 layers (separate pools), H=4, d=128, N_max=8320",
+            "ms_per_layer": round(ms_layer, 4), "new_tokens_per_s": round(T / (ms_layer * 1e-3), 1),
+            "splits": splits,
+            "roofline": {"kernel": "attn_sm100_kernel (paged)", "bound": "hbm", "achieved": round(achieved, 1),
+                         "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                         "frac": round(achieved / float(peaks["hbm_gbs"]), 4),
+                         "peak_source": f"{kind} hbm_gbs", "bytes_per_launch": alg_bytes,
+                         "launch_ms": round(attn_ms, 4), "traffic": None}}
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle on the host cores
+# ----------------------------------------------------------------------------
+
+def run_reference(args):
+    import oracle
+    oracle.build()
+    b0 = synth.workload_attention(args.workload, layer=0)
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for s in range(args.warmup + args.steps):
+        dt, flops, nrows = oracle_sample(b0, per_step, seed=s)
+        if s >= args.warmup:
+            vals.append((dt, flops, nrows))
+    dt = sum(v[0] for v in vals)
+    flops = sum(v[1] for v in vals)
+    rows = sum(v[2] for v in vals)
+    value = flops / dt / 1e12
+    cores = oracle.num_threads()
+    return {
+        "impl": "reference",
+        "metric": "HSTU attention fwd TFLOP/s + tokens/s, % of B200 BF16 peak / HBM BW",
+        "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; no dataset)",
+        "config": {"workload": f"{args.workload}: 8-layer HSTU attention, B={b0.batch}, T={b0.total_tokens}, "
+                               f"H=4, d=128, N_max={b0.n_max}", "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} random query rows of layer 0 (all heads), fp64 C oracle"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="stack8_bf16", choices=["stack8_bf16", "stack8_n8192"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-paged", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="fewer layers (profiling captures only; the bench line uses all 8)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    from generative_recommender_attention_jagged_b200 import build as hbuild
+    hbuild.build()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    result, b0 = run_ours(args, rank, world, device)
+    if rank == 0 and not args.no_paged and world == 1:
+        result["paged"] = run_paged_bench(args, device)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        dt, flops, nrows = oracle_sample(b0, 12.0)
+        result["cpu_baseline"] = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                                  "kind": "oracle",
+                                  "sample": f"{nrows} random query rows of layer 0 (all 4 heads), fp64 C oracle, "
+                                            f"{dt:.1f} s"}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -343,3 +343,35 @@ def workload_stack(workload: str, num_layers: Optional[int] = None,
                        num_candidates=None if cand is None else cand.astype(np.int32),
                        layers=[(rp, rt, w) for (rp, rt), w in zip(rabs, weights)],
                        n_max=n_max, num_heads=H, head_dim=d, d_model=dm, alpha=1.0 / math.sqrt(d))
+
+
+def attention_stack(workload: str, num_layers: Optional[int] = None, seed: Optional[int] = None):
+    """Attention inputs of every layer of a stack: one set of users, lengths and
+    timestamps (drawn from the layer-0 stream), per-layer rab tables and
+    Q/K/V/U (drawn from each layer's own stream)."""
+    base = workload_attention(workload, layer=0, seed=seed)
+    layers = {"stack8_bf16": 8, "stack8_n8192": 8, "mfalcon_bf16": 2, "layer_bf16": 1, "tiny_fp32": 1}
+    L = layers[workload] if num_layers is None else num_layers
+    out = [base]
+    T, H, d = base.q.shape
+    for layer in range(1, L):
+        rng = _rng(workload, layer, seed)
+        rab_pos, rab_ts = draw_rab(rng, base.n_max)
+        q = draw_normal(rng, (T, H, d), 1.0, base.q.dtype)
+        k = draw_normal(rng, (T, H, d), 1.0, base.q.dtype)
+        v = draw_normal(rng, (T, H, d), 1.0, base.q.dtype)
+        u = draw_normal(rng, (T, H * d), 1.0, base.q.dtype)
+        out.append(dataclasses.replace(base, q=q, k=k, v=v, u=u, rab_pos=rab_pos, rab_ts=rab_ts))
+    return out
+
+
+def paged_stack(num_layers: int = 8, seed: Optional[int] = None):
+    """The paged workload of every layer: one set of users and cached lengths,
+    a separate page pool and page table per layer."""
+    rng0 = _rng("paged_bf16", 0, seed)
+    cached = rng0.integers(6144, 8192, size=8, endpoint=True)
+    out = []
+    for layer in range(num_layers):
+        rng = _rng("paged_bf16", 100 + layer, seed)
+        out.append(paged_batch(cached, 64, 64, 4, 128, 8320, rng=rng))
+    return out
