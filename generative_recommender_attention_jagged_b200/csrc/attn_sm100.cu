@@ -1,15 +1,17 @@
 // HSTU pointwise attention on the sm_100a tensor cores (bf16 in, fp32 accumulate).
 //
-// One CTA computes one work item: 128 query rows of one (user, head) against
-// a range of 128-key tiles (all the tiles the rows need, or one split of them
-// in paged mode).  Per key tile:
+// One CTA computes one work item: two 128-row query tiles A and B (rows
+// qs..qs+255 of one user and head) against a range of 128-key tiles (all the
+// tiles the rows need, or one split of them in paged mode).  Per key tile and
+// query tile X:
 //
-//   S  = Q K^T            tcgen05.mma, A = Q (smem, K-major), B = K (smem, K-major),
-//                         fp32 accumulator in tensor memory (128 lanes x 128 columns)
-//   P  = SiLU(alpha S + rab_pos[p_i - p_j + N - 1] + rab_ts[bucket(t_i - t_j)]),
-//        0 outside the allowed set; computed by four elementwise warps that read
-//        S with tcgen05.ld and write P as bf16 pairs back over S (tcgen05.st)
-//   O += P V              tcgen05.mma, A = P (tensor memory), B = V (smem, MN-major)
+//   S_X  = Q_X K^T          tcgen05.mma, A = Q_X (smem, K-major), B = K (smem,
+//                           K-major), fp32 accumulator in tensor memory
+//   P_X  = SiLU(alpha S_X + rab_pos[p_i - p_j + N - 1] + rab_ts[bucket(t_i - t_j)]),
+//          0 outside the allowed set; computed by the elementwise warpgroup of
+//          X, which reads S_X with tcgen05.ld and writes P_X as bf16 pairs back
+//          over S_X (tcgen05.st)
+//   O_X += P_X V            tcgen05.mma, A = P_X (tensor memory), B = V (smem, MN-major)
 //
 // There is no softmax, no row maximum and no rescaling: the weights are
 // pointwise ("Generative Recommenders at Scale", Inside NVIDIA's GPU-native
@@ -20,22 +22,26 @@
 // the candidate's own term a_ii v_i is added by the epilogue, so no tile of
 // the candidate x candidate block is ever issued.
 //
-// Warp roles (192 threads): warps 0-3 elementwise (thread = query row = TMEM
-// lane), warp 4 TMA producer (Q once, K/V through a 2-stage ring, paged
-// prefix gathered page by page), warp 5 MMA issuer and TMEM owner.  S is
-// double-buffered in tensor memory so QK^T of tile t+1 runs while the
-// elementwise warps turn tile t into P.  Every wait is bounded (about 2 s),
-// after which the kernel reports HSTU_ERR_TIMEOUT and winds down.
+// Warp roles (320 threads): warps 0-3 elementwise for tile A, warps 4-7 for
+// tile B (thread = query row = TMEM lane), warp 8 producer (Q once; K/V
+// through a 2-stage ring by TMA, the paged prefix page by page; per key tile
+// it also stages the keys' timestamps and a window of 0.5*rab_pos in shared
+// memory), warp 9 MMA issuer and TMEM owner.  Tensor memory holds S_A, S_B,
+// O_A, O_B (4 x 128 columns); while one warpgroup turns S into P the tensor
+// core runs the other tile's GEMMs.  Every wait is bounded (about 2 s), after
+// which the kernel reports HSTU_ERR_TIMEOUT and winds down.
 //
-// Time buckets are exact: the elementwise thread finds the bucket of its
-// row's first key by a binary search over integer edges, then walks down the
-// edges as the keys get closer in time (timestamps are non-decreasing inside
-// a user, so |t_i - t_j| only shrinks along a row); warps whose rows stay in
-// one bucket over the whole tile skip the walk.
+// Elementwise work per score: hb = s/2 = (alpha/2) S + 0.5 (rab_pos + rab_ts)
+// with packed f32x2 FMA, SiLU(s) = hb (1 + tanh hb) with one MUFU tanh.  Time
+// buckets are exact: a thread finds the bucket of its row's first key once per
+// work item by a binary search over integer edges, then walks down the edges
+// as the keys come closer in time (timestamps are non-decreasing inside a
+// user, so |t_i - t_j| only shrinks along a row).  One compare per tile tells
+// whether a row stays in its bucket over the whole tile; warps where every row
+// does skip the walk, and the walk runs as its own pass so that the SiLU loop
+// stays branch-free.
 #include <cuda_bf16.h>
 #include <stdint.h>
-
-#include <algorithm>
 
 #include "device_common.cuh"
 
@@ -43,33 +49,43 @@ namespace hstu {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kQTiles = 2;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr int kTileBytes = kTile * 128 * 2;  // 128 rows x 128 bf16 = 32 KB
 constexpr int kHalfBytes = kTile * 128;      // 128 rows x 64 bf16: one 128B-swizzled box
-constexpr uint32_t kTmemCols = 512;          // S0 [0,128) S1 [128,256) O [256,384)
+constexpr uint32_t kTmemCols = 512;          // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
 constexpr int kHeadDim = 128;
+constexpr int kWin = 384;                    // position-bias window of a 256-row x 128-key block
+
+struct Meta {
+  long long ts[kTile];      // key timestamps of the tile (the last one repeated past its width)
+  float win[4][kWin];       // reversed window of 0.5*rab_pos, four copies shifted by 0..3 floats
+};
 
 struct __align__(1024) Smem {
-  uint8_t q[kTileBytes];
+  uint8_t q[kQTiles][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
+  Meta meta[kStages];
   long long thr[kMaxBuckets];
   float rab_ts_half[kMaxBuckets];
-  long long ts_tile[2][kTile];
-  float win[2][256];
   uint64_t bar_q;
   uint64_t bar_k_full[kStages];
   uint64_t bar_v_full[kStages];
+  uint64_t bar_meta_full[kStages];
   uint64_t bar_kv_empty[kStages];
-  uint64_t bar_s_full[2];
-  uint64_t bar_p_full[2];
+  uint64_t bar_s_full[kQTiles];
+  uint64_t bar_p_full[kQTiles];
   uint64_t bar_o_full;
   uint32_t tmem_base;
   int abort;
 };
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
   uint4 r;
@@ -84,16 +100,99 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-// elementwise warps agree on a flag (bar.red.and over the 128 threads)
-__device__ __forceinline__ bool ew_all(bool ok) {
+__device__ __forceinline__ float4 lds_f4(const float* p) {
+  float4 r;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "r"(smem_u32(p)));
+  return r;
+}
+
+// the 128 threads of one elementwise warpgroup agree on a flag
+__device__ __forceinline__ bool ew_all(bool ok, int group) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      "bar.red.and.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)ok)
+      : "r"((uint32_t)ok), "r"(1 + group)
       : "memory");
   return r != 0;
+}
+
+// packed fp32 pairs (sm_100): lo in the low half
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// Row state of the exact time-bucket walk.
+struct Walk {
+  long long t_i;   // the row's timestamp
+  long long tlim;  // bucket b still holds while t_j <= tlim  (tlim = t_i + 1 - thr[b])
+  int b;
+  float tsb;       // 0.5 * rab_ts[b]
+};
+
+__device__ __forceinline__ void walk_to(Walk& w, long long tj, const long long* thr, const float* rts) {
+  while (w.b > 0 && tj > w.tlim) {
+    --w.b;
+    w.tlim = w.t_i + 1 - thr[w.b];
+    w.tsb = rts[w.b];
+  }
+}
+
+// 32 scores of one row: S (fp32 bits) -> P (bf16 pairs).  WALK: per-column
+// time bias from the walk; MASK: zero the columns past climit.
+template <bool WALK, bool MASK>
+__device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&pk)[16], const float* wp,
+                                           const long long* ts, int col0, int climit, float alpha_half,
+                                           Walk& w, const long long* thr, const float* rts) {
+  float tsv[32];
+  if constexpr (WALK) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      walk_to(w, ts[col0 + c], thr, rts);
+      tsv[c] = w.tsb;
+    }
+  }
+  const uint64_t ah2 = pk2(alpha_half, alpha_half);
+  const uint64_t tsb2 = pk2(w.tsb, w.tsb);
+#pragma unroll
+  for (int c4 = 0; c4 < 8; ++c4) {
+    const float4 w4 = lds_f4(wp + col0 + 4 * c4);
+#pragma unroll
+    for (int hlf = 0; hlf < 2; ++hlf) {
+      const int c = 4 * c4 + 2 * hlf;
+      uint64_t bias2 = hlf == 0 ? pk2(w4.x, w4.y) : pk2(w4.z, w4.w);
+      bias2 = add2(bias2, WALK ? pk2(tsv[c], tsv[c + 1]) : tsb2);
+      const uint64_t h2 = fma2(pk2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), ah2, bias2);
+      float h0, h1;
+      upk2(h2, h0, h1);
+      const uint64_t p2 = fma2(h2, pk2(tanh_approx(h0), tanh_approx(h1)), h2);  // hb (1 + tanh hb)
+      float p0, p1;
+      upk2(p2, p0, p1);
+      if constexpr (MASK) {
+        p0 = (col0 + c <= climit) ? p0 : 0.f;
+        p1 = (col0 + c + 1 <= climit) ? p1 : 0.f;
+      }
+      pk[c >> 1] = pack_bf16x2(p0, p1);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -110,25 +209,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   // a work list not written by this call's scheduler must not send us out of bounds
   if (it.user < 0 || it.user >= a.B || it.head < 0 || it.head >= a.H || it.split < 0 ||
       it.split >= a.num_splits || it.qtile < 0 ||
-      it.qtile * kTile >= a.q_offsets[it.user + 1] - a.q_offsets[it.user])
+      it.qtile * kQTiles * kTile >= a.q_offsets[it.user + 1] - a.q_offsets[it.user])
     return;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const TileGeom g = tile_geom(a, it.user, it.qtile);
+  const TileGeom gA = tile_geom(a, it.user, it.qtile * kQTiles);
+  const bool hasB = (it.qtile * kQTiles + 1) * kTile < a.q_offsets[it.user + 1] - a.q_offsets[it.user];
+  const TileGeom gB = hasB ? tile_geom(a, it.user, it.qtile * kQTiles + 1) : gA;
+  const int nA = gA.n_tiles;
+  const int nB = hasB ? gB.n_tiles : 0;
   int tb, te;
-  split_range(g.n_tiles, it.split, a.num_splits, tb, te);
-  const int nt = te - tb;
+  split_range(max(nA, nB), it.split, a.num_splits, tb, te);
+  const int cA = max(0, min(te, nA) - tb);  // key tiles of this item for tile A
+  const int cB = max(0, min(te, nB) - tb);
+  const int cT = max(cA, cB);
+  const int prmin = min(gA.qs, gA.h);       // smallest query position of the item
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.bar_k_full[s], 1);
       mbar_init(&sm.bar_v_full[s], 1);
+      mbar_init(&sm.bar_meta_full[s], 32);
       mbar_init(&sm.bar_kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.bar_s_full[b], 1);
-      mbar_init(&sm.bar_p_full[b], kTile);
+    for (int x = 0; x < kQTiles; ++x) {
+      mbar_init(&sm.bar_s_full[x], 1);
+      mbar_init(&sm.bar_p_full[x], kTile);
     }
     mbar_init(&sm.bar_o_full, 1);
     sm.abort = 0;
@@ -138,11 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.thr[x] = tab.thr[x];
     sm.rab_ts_half[x] = x < a.nb ? 0.5f * a.rab_ts[x] : 0.f;
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -157,28 +264,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
     const int head = it.head;
     if (lane == 0) {
-      mbar_arrive_expect_tx(&sm.bar_q, kTileBytes);
-      tma_load_3d(sm.q, &tm_q, &sm.bar_q, 0, head, g.qrow0);
-      tma_load_3d(sm.q + kHalfBytes, &tm_q, &sm.bar_q, 64, head, g.qrow0);
+      mbar_arrive_expect_tx(&sm.bar_q, (hasB ? 2 : 1) * kTileBytes);
+      tma_load_3d(sm.q[0], &tm_q, &sm.bar_q, 0, head, gA.qrow0);
+      tma_load_3d(sm.q[0] + kHalfBytes, &tm_q, &sm.bar_q, 64, head, gA.qrow0);
+      if (hasB) {
+        tma_load_3d(sm.q[1], &tm_q, &sm.bar_q, 0, head, gB.qrow0);
+        tma_load_3d(sm.q[1] + kHalfBytes, &tm_q, &sm.bar_q, 64, head, gB.qrow0);
+      }
     }
-    const int row_base = a.q_offsets[it.user] - g.L;  // row of key position p is row_base + p (p >= L)
+    const int row_base = a.q_offsets[it.user] - gA.L;  // row of key position p is row_base + p (p >= L)
+    const int n_rab = 2 * a.n_max - 1;
     int issued = 0;
-    for (int t = 0; t < nt; ++t) {
+    for (int t = 0; t < cT; ++t) {
       const int s = t % kStages;
       const uint32_t ph = (t / kStages) & 1;
       int k0, width;
-      key_tile(g, tb + t, k0, width);
+      key_tile(gA, tb + t, k0, width);
       bool ok = true;
       if (lane == 0) ok = mbar_wait(&sm.bar_kv_empty[s], ph ^ 1, abort_flag, a.hdr, 1);
       ok = __shfl_sync(~0u, ok, 0);
       if (!ok) break;
       uint8_t* kd = sm.k[s];
       uint8_t* vd = sm.v[s];
-      if (k0 >= g.L) {
+      if (k0 >= gA.L) {
         if (lane == 0) {
           const int row = row_base + k0;
           mbar_arrive_expect_tx(&sm.bar_k_full[s], kTileBytes);
@@ -198,8 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t* prow = a.page_table + (size_t)it.user * a.max_pages + first_page;
         if (man_lo < kTile) {
           const int pid = (width > man_lo) ? prow[full_pages] : 0;
-          const uint8_t* kpage = static_cast<const uint8_t*>(a.k_pool) + ((size_t)pid * a.H + head) * P * kHeadDim * 2;
-          const uint8_t* vpage = static_cast<const uint8_t*>(a.v_pool) + ((size_t)pid * a.H + head) * P * kHeadDim * 2;
+          const uint8_t* kpage =
+              static_cast<const uint8_t*>(a.k_pool) + ((size_t)pid * a.H + head) * P * kHeadDim * 2;
+          const uint8_t* vpage =
+              static_cast<const uint8_t*>(a.v_pool) + ((size_t)pid * a.H + head) * P * kHeadDim * 2;
           const uint32_t kbase = smem_u32(kd), vbase = smem_u32(vd);
           for (int idx = lane; idx < (kTile - man_lo) * 16; idx += 32) {
             const int r = man_lo + (idx >> 4);
@@ -233,6 +347,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // per-tile metadata: key timestamps and the position-bias window
+      Meta& m = sm.meta[s];
+      for (int c = lane; c < kTile; c += 32) m.ts[c] = a.ts[gA.tso + k0 + min(c, width - 1)];
+      const int wb = prmin - k0 - 127 + a.n_max - 1;  // rab_pos index of window entry x = 0
+      for (int z = lane; z < kWin; z += 32) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const int idx = wb + (kWin - 1) - z - p;  // copy p, entry z holds window entry 383 - z - p
+          m.win[p][z] = (idx >= 0 && idx < n_rab) ? 0.5f * __ldg(a.rab_pos + idx) : 0.f;
+        }
+      }
+      mbar_arrive(&sm.bar_meta_full[s]);
       issued = t + 1;
     }
     // no copy may still be landing in shared memory when the CTA exits
@@ -245,47 +371,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, 128, 0, 1);
-      const uint32_t q_base = smem_u32(sm.q);
-      const uint32_t o_tmem = tmem + 256;
-      bool ok = nt == 0 || mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 2);
+      const int cnt[kQTiles] = {cA, cB};
+      auto issue_s = [&](int x, int t) {
+        const uint32_t q_base = smem_u32(sm.q[x]);
+        const uint32_t k_base = smem_u32(sm.k[t % kStages]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          mma_ss(tmem + x * 128, sw128_desc(q_base + off, 16, 1024), sw128_desc(k_base + off, 16, 1024),
+                 idesc_qk, kk > 0);
+        }
+        mma_commit(&sm.bar_s_full[x]);
+      };
+      auto issue_pv = [&](int x, int t) {
+        const uint32_t v_base = smem_u32(sm.v[t % kStages]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, sw128_desc(v_base + kk * 2048, kHalfBytes, 1024),
+                 idesc_pv, (t > 0 || kk > 0));
+      };
+      bool ok = cT == 0 || mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 2);
+      if (ok && cT > 0) ok = mbar_wait(&sm.bar_k_full[0], 0, abort_flag, a.hdr, 3);
       tc_fence_after();
-      for (int t = 0; ok && t <= nt; ++t) {
-        if (t < nt) {
-          const int s = t % kStages;
-          const int buf = t & 1;
-          ok = mbar_wait(&sm.bar_k_full[s], (t / kStages) & 1, abort_flag, a.hdr, 3);
+      if (ok && cT > 0) {
+        for (int x = 0; x < kQTiles; ++x)
+          if (cnt[x] > 0) issue_s(x, 0);
+      }
+      for (int t = 0; ok && t < cT; ++t) {
+        const int s = t % kStages;
+        bool v_ready = false, k_next_ready = false;
+        for (int x = 0; ok && x < kQTiles; ++x) {
+          if (t >= cnt[x]) continue;
+          ok = mbar_wait(&sm.bar_p_full[x], t & 1, abort_flag, a.hdr, 4);
+          if (ok && !v_ready) ok = v_ready = mbar_wait(&sm.bar_v_full[s], (t / kStages) & 1, abort_flag, a.hdr, 5);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t k_base = smem_u32(sm.k[s]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            mma_ss(tmem + buf * 128, sw128_desc(q_base + off, 16, 1024), sw128_desc(k_base + off, 16, 1024),
-                   idesc_qk, kk > 0);
+          issue_pv(x, t);
+          if (t + 1 < cnt[x]) {
+            if (!k_next_ready)
+              ok = k_next_ready = mbar_wait(&sm.bar_k_full[(t + 1) % kStages], ((t + 1) / kStages) & 1,
+                                            abort_flag, a.hdr, 3);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(x, t + 1);
           }
-          mma_commit(&sm.bar_s_full[buf]);
         }
-        if (t > 0) {
-          const int tp = t - 1;
-          const int sp = tp % kStages;
-          const int bp = tp & 1;
-          ok = mbar_wait(&sm.bar_p_full[bp], (tp >> 1) & 1, abort_flag, a.hdr, 4);
-          if (!ok) break;
-          ok = mbar_wait(&sm.bar_v_full[sp], (tp / kStages) & 1, abort_flag, a.hdr, 5);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t v_base = smem_u32(sm.v[sp]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(o_tmem, tmem + bp * 128 + kk * 8, sw128_desc(v_base + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                   (tp > 0 || kk > 0));
-          mma_commit(&sm.bar_kv_empty[sp]);
-        }
+        if (ok) mma_commit(&sm.bar_kv_empty[s]);
       }
       mma_commit(&sm.bar_o_full);
       // tensor memory is freed below only after every issued MMA completed
@@ -294,102 +430,88 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ elementwise
-    const int r = threadIdx.x;  // query row of the tile == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const bool valid = r < g.nq_rows;
+    const int x = warp >> 2;                 // query tile of this warpgroup
+    const int r = threadIdx.x & (kTile - 1); // query row of the tile == TMEM lane
+    const TileGeom& g = x == 0 ? gA : gB;
+    const int cnt = x == 0 ? cA : cB;
+    const bool exists = x == 0 || hasB;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const bool valid = exists && r < g.nq_rows;
     const int i = min(g.qs + r, g.n - 1);  // rows past the user repeat its last row (discarded)
     const int jmax = i < g.h ? i : g.h - 1;
     const int pr = min(i, g.h);
-    const int pr_min = min(g.qs, g.h);
-    const int xoff = pr - pr_min + 127;
-    const long long t_i = a.ts[g.tso + i];
+    const int y0 = 256 - (pr - prmin);     // window entry of column 0 (reversed window)
+    const int wcopy = y0 & 3;
+    const int woff = y0 - wcopy;
     const float alpha_half = 0.5f * a.alpha;
-    const int n_rab = 2 * a.n_max - 1;
+    const uint32_t s_tmem = tmem + lane_base + x * 128;
+    Walk w;
+    w.t_i = a.ts[g.tso + i];
+    w.b = 0;
+    w.tlim = 0;
+    w.tsb = 0.f;
     bool ok = true;
-    for (int t = 0; t < nt; ++t) {
-      const int buf = t & 1;
+    for (int t = 0; t < cnt; ++t) {
+      const int s = t % kStages;
       int k0, width;
       key_tile(g, tb + t, k0, width);
-      sm.ts_tile[buf][r] = a.ts[g.tso + k0 + min(r, width - 1)];
-      const int wb = pr_min - k0 - 127 + a.n_max - 1;
-      for (int x = r; x < 256; x += kTile) {
-        const int idx = wb + x;
-        sm.win[buf][x] = (idx >= 0 && idx < n_rab) ? 0.5f * a.rab_pos[idx] : 0.f;
-      }
-      ok = mbar_wait(&sm.bar_s_full[buf], (t >> 1) & 1, abort_flag, a.hdr, 6);
-      ok = ew_all(ok);  // also publishes ts_tile / win to the other elementwise warps
+      ok = mbar_wait(&sm.bar_meta_full[s], (t / kStages) & 1, abort_flag, a.hdr, 6);
+      ok = ok && mbar_wait(&sm.bar_s_full[x], t & 1, abort_flag, a.hdr, 6);
+      ok = ew_all(ok, x);
       if (!ok) break;
       tc_fence_after();
+      const Meta& m = sm.meta[s];
       const int climit = min(jmax - k0, width - 1);  // columns c <= climit are allowed
-      const bool need_mask = !__all_sync(~0u, climit >= kTile - 1);
-      int b = 0;
-      bool uni = true;
-      if (climit >= 0) {
-        b = bucket_of_dt(sm.thr, t_i - sm.ts_tile[buf][0]);
-        uni = b == bucket_of_dt(sm.thr, t_i - sm.ts_tile[buf][climit]);
+      if (t == 0) {
+        w.b = bucket_of_dt(sm.thr, w.t_i - m.ts[0]);
+        w.tlim = w.t_i + 1 - sm.thr[w.b];
+        w.tsb = sm.rab_ts_half[w.b];
       }
+      const bool uni = m.ts[max(0, climit)] <= w.tlim;  // no bucket edge before the last allowed key
       const bool walk = !__all_sync(~0u, uni);
-      float tsb = sm.rab_ts_half[b];
-      long long tlim = t_i + 1 - sm.thr[b];  // bucket drops once t_j > tlim
-      const long long* tst = sm.ts_tile[buf];
-      const float* win = sm.win[buf];
-      const uint32_t s_tmem = tmem + lane_base + buf * 128;
+      const bool need_mask = !__all_sync(~0u, climit >= kTile - 1);
+      const float* wp = &m.win[wcopy][woff];
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t sr[32];
         tmem_ld32(s_tmem + ch * 32, sr);
         tmem_wait_ld();
         uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = ch * 32 + c + e;
-            if (walk) {
-              const long long tj = tst[col];
-              while (b > 0 && tj > tlim) {
-                --b;
-                tlim = t_i + 1 - sm.thr[b];
-                tsb = sm.rab_ts_half[b];
-              }
-            }
-            const float hb = fmaf(__uint_as_float(sr[c + e]), alpha_half, win[xoff - col] + tsb);
-            const float th = tanh_approx(hb);
-            float p = fmaf(hb, th, hb);  // SiLU(s) with hb = s/2: hb (1 + tanh hb)
-            if (need_mask) p = (col <= climit) ? p : 0.f;
-            pv[e] = p;
-          }
-          pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
+        if (walk) {
+          if (need_mask) silu_chunk<true, true>(sr, pk, wp, m.ts, ch * 32, climit, alpha_half, w, sm.thr, sm.rab_ts_half);
+          else silu_chunk<true, false>(sr, pk, wp, m.ts, ch * 32, climit, alpha_half, w, sm.thr, sm.rab_ts_half);
+        } else {
+          if (need_mask) silu_chunk<false, true>(sr, pk, wp, m.ts, ch * 32, climit, alpha_half, w, sm.thr, sm.rab_ts_half);
+          else silu_chunk<false, false>(sr, pk, wp, m.ts, ch * 32, climit, alpha_half, w, sm.thr, sm.rab_ts_half);
         }
         tmem_st16(s_tmem + ch * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.bar_p_full[buf]);
+      mbar_arrive(&sm.bar_p_full[x]);
     }
-    if (ok && nt > 0) {
-      ok = ew_all(mbar_wait(&sm.bar_o_full, 0, abort_flag, a.hdr, 7));
+    if (ok && cT > 0) {
+      ok = ew_all(mbar_wait(&sm.bar_o_full, 0, abort_flag, a.hdr, 7), x);
       tc_fence_after();
     }
-    if (ok) {
+    if (ok && exists) {
       float* orow = a.o_ws + (((size_t)it.split * a.T_q + (g.qrow0 + r)) * a.H + it.head) * kHeadDim;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t orr[32];
-        if (nt > 0) {
-          tmem_ld32(tmem + lane_base + 256 + ch * 32, orr);
+        if (cnt > 0) {
+          tmem_ld32(tmem + lane_base + 256 + x * 128 + ch * 32, orr);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) orr[x] = 0u;
+          for (int e = 0; e < 32; ++e) orr[e] = 0u;
         }
         if (valid) {
           float4* dst = reinterpret_cast<float4*>(orow + ch * 32);
 #pragma unroll
-          for (int x = 0; x < 8; ++x)
-            dst[x] = make_float4(__uint_as_float(orr[4 * x]), __uint_as_float(orr[4 * x + 1]),
-                                 __uint_as_float(orr[4 * x + 2]), __uint_as_float(orr[4 * x + 3]));
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(orr[4 * e]), __uint_as_float(orr[4 * e + 1]),
+                                 __uint_as_float(orr[4 * e + 2]), __uint_as_float(orr[4 * e + 3]));
         }
       }
     }
@@ -398,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
@@ -406,12 +528,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_attn_sm100(const AttnArgs& a, const BucketTable& thr, const CUtensorMap& tm_q,
                               const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_kpool,
                               const CUtensorMap& tm_vpool, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static unsigned long long attr_set = 0;  // one bit per device
+  if (dev < 64 && !(attr_set & (1ull << dev))) {
     cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set |= 1ull << dev;
   }
   if (a.max_items <= 0) return cudaSuccess;
   attn_sm100_kernel<<<a.max_items, kThreads, kSmemBytes, s>>>(a, thr, tm_q, tm_k, tm_v, tm_kpool, tm_vpool);

@@ -113,7 +113,7 @@ struct Layout {
 Layout layout_for(const hstu_attn_params* p, int splits, bool tc) {
   Layout l;
   const long long T = p->total_tokens;
-  const long long qtiles = (T + kTile - 1) / kTile + p->batch;  // sum_u ceil(n_u/128) <= T/128 + B
+  const long long qtiles = (T + kItemRows - 1) / kItemRows + p->batch;  // sum_u ceil(n_u/256) <= T/256 + B
   const long long items = tc ? qtiles * p->num_heads * splits : 0;
   l.max_items = (int)items;
   l.items_off = sizeof(WsHeader);
@@ -256,7 +256,7 @@ int32_t hstu_attn_paged_default_splits(const hstu_attn_params* p, int32_t max_ca
   if (check_params(p) != HSTU_OK) return 1;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long qtiles = (p->total_tokens + kTile - 1) / kTile;
+  const long long qtiles = (p->total_tokens + kItemRows - 1) / kItemRows;
   const long long units = std::max<long long>(1, qtiles * p->num_heads);
   const long long key_tiles = std::max(1, (max_cached_len + kTile - 1) / kTile);
   long long s = (sms + units - 1) / units;          // at least one wave of CTAs

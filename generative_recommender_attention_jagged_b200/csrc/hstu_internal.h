@@ -10,6 +10,7 @@ namespace hstu {
 
 constexpr int kMaxBuckets = 128;   // rab_ts entries supported
 constexpr int kTile = 128;         // query rows / key rows per tensor-core tile
+constexpr int kItemRows = 256;     // query rows per tensor-core work item (two tiles)
 constexpr int kMaxSplits = 64;
 
 // Bucket edges: thr[b] = smallest integer x with ln(x) >= 0.301*b, for
@@ -32,10 +33,10 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header size");
 
-// Work item: one (user, query tile, head, key split).
+// Work item: one (user, block of kItemRows query rows, head, key split).
 struct WorkItem {
   int32_t user;
-  int32_t qtile;
+  int32_t qtile;  // index of the kItemRows-row block inside the user's query rows
   int32_t head;
   int32_t split;
 };

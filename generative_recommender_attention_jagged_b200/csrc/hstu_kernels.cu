@@ -86,14 +86,18 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const AttnArgs 
     return;
   }
   const int per = a.H * a.num_splits;
+  constexpr int tiles_per_item = kItemRows / kTile;
+  // cost of a block of query rows: key tiles of its longest tile, per split
   auto cost_of = [&](int user, int m) {
-    const TileGeom g = tile_geom(a, user, m);
-    const int c = ceil_div(g.n_tiles, a.num_splits);
-    return min(c, kCostBins - 1);
+    const int nq = a.q_offsets[user + 1] - a.q_offsets[user];
+    int c = 0;
+    for (int x = 0; x < tiles_per_item && (m * tiles_per_item + x) * kTile < nq; ++x)
+      c = max(c, tile_geom(a, user, m * tiles_per_item + x).n_tiles);
+    return min(ceil_div(c, a.num_splits), kCostBins - 1);
   };
   for (int u = tid; u < a.B; u += blockDim.x) {
     const int nq = a.q_offsets[u + 1] - a.q_offsets[u];
-    for (int m = ceil_div(nq, kTile) - 1; m >= 0; --m) atomicAdd(&hist[cost_of(u, m)], per);
+    for (int m = ceil_div(nq, kItemRows) - 1; m >= 0; --m) atomicAdd(&hist[cost_of(u, m)], per);
   }
   __syncthreads();
   // start[c] = number of items with a cost above c (descending order)
@@ -116,7 +120,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const AttnArgs 
   __syncthreads();
   for (int u = tid; u < a.B; u += blockDim.x) {
     const int nq = a.q_offsets[u + 1] - a.q_offsets[u];
-    for (int m = ceil_div(nq, kTile) - 1; m >= 0; --m) {
+    for (int m = ceil_div(nq, kItemRows) - 1; m >= 0; --m) {
       const int pos = atomicAdd(&start[cost_of(u, m)], per);
       for (int h = 0; h < a.H; ++h)
         for (int s = 0; s < a.num_splits; ++s) {
