@@ -36,10 +36,13 @@
 // buckets are exact: a thread finds the bucket of its row's first key once per
 // work item by a binary search over integer edges, then walks down the edges
 // as the keys come closer in time (timestamps are non-decreasing inside a
-// user, so |t_i - t_j| only shrinks along a row).  One compare per tile tells
-// whether a row stays in its bucket over the whole tile; warps where every row
-// does skip the walk, and the walk runs as its own pass so that the SiLU loop
-// stays branch-free.
+// user, so |t_i - t_j| only shrinks along a row).  Per 32-column chunk one
+// compare tells whether a row stays in its bucket; a chunk where every row of
+// the warp does uses a constant, a chunk with at most one edge per row finds
+// it by a 5-step search and selects, and only chunks with more edges (next to
+// the diagonal) walk column by column.  The SiLU loop itself is branch-free.
+// The producer loads each tile's metadata into registers one tile ahead, so
+// its global-load latency hides behind the wait for a free stage.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -59,10 +62,11 @@ constexpr int kHalfBytes = kTile * 128;      // 128 rows x 64 bf16: one 128B-swi
 constexpr uint32_t kTmemCols = 512;          // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
 constexpr int kHeadDim = 128;
 constexpr int kWin = 384;                    // position-bias window of a 256-row x 128-key block
+constexpr int kWinStride = kWin + 8;         // copies 32 bytes apart: a warp's 16-byte reads hit 8 bank groups
 
 struct Meta {
-  long long ts[kTile];      // key timestamps of the tile (the last one repeated past its width)
-  float win[4][kWin];       // reversed window of 0.5*rab_pos, four copies shifted by 0..3 floats
+  long long ts[kTile];          // key timestamps of the tile (the last one repeated past its width)
+  float win[4][kWinStride];     // reversed window of 0.5*rab_pos, four copies shifted by 0..3 floats
 };
 
 struct __align__(1024) Smem {
@@ -156,19 +160,28 @@ __device__ __forceinline__ void walk_to(Walk& w, long long tj, const long long* 
   }
 }
 
-// 32 scores of one row: S (fp32 bits) -> P (bf16 pairs).  WALK: per-column
-// time bias from the walk; MASK: zero the columns past climit.
-template <bool WALK, bool MASK>
+// Time-bias modes of a 32-column chunk.
+enum BiasMode { kBiasConst = 0, kBiasEdge = 1, kBiasWalk = 2 };
+
+// 32 scores of one row: S (fp32 bits) -> P (bf16 pairs).
+//   kBiasConst: the row's time bucket is the same over the chunk (w.tsb)
+//   kBiasEdge:  one bucket edge: columns before `pos` use tsb_lo, the rest w.tsb
+//   kBiasWalk:  per-column walk over the bucket edges
+// MASK zeroes the columns past climit.
+template <int MODE, bool MASK>
 __device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&pk)[16], const float* wp,
-                                           const long long* ts, int col0, int climit, float alpha_half,
-                                           Walk& w, const long long* thr, const float* rts) {
+                                           const long long* ts, int col0, int climit, int pos, float tsb_lo,
+                                           float alpha_half, Walk& w, const long long* thr, const float* rts) {
   float tsv[32];
-  if constexpr (WALK) {
+  if constexpr (MODE == kBiasWalk) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
       walk_to(w, ts[col0 + c], thr, rts);
       tsv[c] = w.tsb;
     }
+  } else if constexpr (MODE == kBiasEdge) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) tsv[c] = (col0 + c < pos) ? tsb_lo : w.tsb;
   }
   const uint64_t ah2 = pk2(alpha_half, alpha_half);
   const uint64_t tsb2 = pk2(w.tsb, w.tsb);
@@ -179,7 +192,7 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&
     for (int hlf = 0; hlf < 2; ++hlf) {
       const int c = 4 * c4 + 2 * hlf;
       uint64_t bias2 = hlf == 0 ? pk2(w4.x, w4.y) : pk2(w4.z, w4.w);
-      bias2 = add2(bias2, WALK ? pk2(tsv[c], tsv[c + 1]) : tsb2);
+      bias2 = add2(bias2, MODE == kBiasConst ? tsb2 : pk2(tsv[c], tsv[c + 1]));
       const uint64_t h2 = fma2(pk2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), ah2, bias2);
       float h0, h1;
       upk2(h2, h0, h1);
@@ -193,6 +206,19 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&
       pk[c >> 1] = pack_bf16x2(p0, p1);
     }
   }
+}
+
+template <bool MASK>
+__device__ __forceinline__ void silu_chunk_mode(int mode, const uint32_t (&sr)[32], uint32_t (&pk)[16],
+                                                const float* wp, const long long* ts, int col0, int climit,
+                                                int pos, float tsb_lo, float alpha_half, Walk& w,
+                                                const long long* thr, const float* rts) {
+  if (mode == kBiasConst)
+    silu_chunk<kBiasConst, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts);
+  else if (mode == kBiasEdge)
+    silu_chunk<kBiasEdge, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts);
+  else
+    silu_chunk<kBiasWalk, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -278,6 +304,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int row_base = a.q_offsets[it.user] - gA.L;  // row of key position p is row_base + p (p >= L)
     const int n_rab = 2 * a.n_max - 1;
+    // Per-tile metadata (key timestamps, position-bias window) is loaded into
+    // registers one tile ahead, so its global-load latency hides behind the
+    // wait for a free stage.  Lane l holds timestamps of columns l + 32k and
+    // window entries x = l + 32k - 3 (x in [-3, 384)).
+    constexpr int kWinLoads = (kWin + 3 + 31) / 32;
+    long long mts[4];
+    float mwin[kWinLoads];
+    auto load_meta = [&](int t) {
+      int k0, width;
+      key_tile(gA, tb + t, k0, width);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mts[k] = a.ts[gA.tso + k0 + min(lane + 32 * k, width - 1)];
+      const int wb = prmin - k0 - 127 + a.n_max - 1;  // rab_pos index of window entry x = 0
+#pragma unroll
+      for (int k = 0; k < kWinLoads; ++k) {
+        const int idx = wb + lane + 32 * k - 3;
+        mwin[k] = (idx >= 0 && idx < n_rab) ? 0.5f * __ldg(a.rab_pos + idx) : 0.f;
+      }
+    };
+    if (cT > 0) load_meta(0);
     int issued = 0;
     for (int t = 0; t < cT; ++t) {
       const int s = t % kStages;
@@ -347,18 +393,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // per-tile metadata: key timestamps and the position-bias window
+      // publish this tile's metadata, then start loading the next tile's
       Meta& m = sm.meta[s];
-      for (int c = lane; c < kTile; c += 32) m.ts[c] = a.ts[gA.tso + k0 + min(c, width - 1)];
-      const int wb = prmin - k0 - 127 + a.n_max - 1;  // rab_pos index of window entry x = 0
-      for (int z = lane; z < kWin; z += 32) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) m.ts[lane + 32 * k] = mts[k];
+#pragma unroll
+      for (int k = 0; k < kWinLoads; ++k) {
+        const int x = lane + 32 * k - 3;  // copy p, entry z holds window entry 383 - z - p
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-          const int idx = wb + (kWin - 1) - z - p;  // copy p, entry z holds window entry 383 - z - p
-          m.win[p][z] = (idx >= 0 && idx < n_rab) ? 0.5f * __ldg(a.rab_pos + idx) : 0.f;
+          const int z = (kWin - 1) - x - p;
+          if (z >= 0 && z < kWin) m.win[p][z] = mwin[k];
         }
       }
       mbar_arrive(&sm.bar_meta_full[s]);
+      if (t + 1 < cT) load_meta(t + 1);
       issued = t + 1;
     }
     // no copy may still be landing in shared memory when the CTA exits
@@ -467,23 +516,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         w.tlim = w.t_i + 1 - sm.thr[w.b];
         w.tsb = sm.rab_ts_half[w.b];
       }
-      const bool uni = m.ts[max(0, climit)] <= w.tlim;  // no bucket edge before the last allowed key
-      const bool walk = !__all_sync(~0u, uni);
       const bool need_mask = !__all_sync(~0u, climit >= kTile - 1);
       const float* wp = &m.win[wcopy][woff];
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t sr[32];
         tmem_ld32(s_tmem + ch * 32, sr);
-        tmem_wait_ld();
-        uint32_t pk[16];
-        if (walk) {
-          if (need_mask) silu_chunk<true, true>(sr, pk, wp, m.ts, ch * 32, climit, alpha_half, w, sm.thr, sm.rab_ts_half);
-          else silu_chunk<true, false>(sr, pk, wp, m.ts, ch * 32, climit, alpha_half, w, sm.thr, sm.rab_ts_half);
-        } else {
-          if (need_mask) silu_chunk<false, true>(sr, pk, wp, m.ts, ch * 32, climit, alpha_half, w, sm.thr, sm.rab_ts_half);
-          else silu_chunk<false, false>(sr, pk, wp, m.ts, ch * 32, climit, alpha_half, w, sm.thr, sm.rab_ts_half);
+        // time-bias mode of this chunk (decided while the TMEM load is in flight):
+        // the walk state always describes the last column processed so far
+        const int col0 = ch * 32;
+        const int col_last = min(col0 + 31, climit);
+        const bool none = col_last < col0;                    // chunk fully masked for this row
+        const long long t_last = m.ts[max(col_last, 0)];
+        const bool uni = none || t_last <= w.tlim;            // no bucket edge in the chunk
+        int mode = kBiasConst, pos = col0 + 32;
+        float tsb_lo = w.tsb;
+        if (!__all_sync(~0u, uni)) {
+          const long long tlim2 = w.b > 0 ? w.t_i + 1 - sm.thr[w.b - 1] : LLONG_MIN;
+          const bool one = uni || t_last <= tlim2;              // at most one edge in the chunk
+          if (__all_sync(~0u, one)) {
+            mode = kBiasEdge;
+            if (!uni) {
+              // first column of the chunk past the edge (timestamps are sorted)
+              pos = col0;
+#pragma unroll
+              for (int step = 16; step >= 1; step >>= 1)
+                if (m.ts[pos + step - 1] <= w.tlim) pos += step;
+              --w.b;
+              w.tlim = tlim2;
+              w.tsb = sm.rab_ts_half[w.b];
+            }
+          } else {
+            mode = kBiasWalk;
+          }
         }
+        tmem_wait_ld(sr);
+        uint32_t pk[16];
+        if (need_mask)
+          silu_chunk_mode<true>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w, sm.thr, sm.rab_ts_half);
+        else
+          silu_chunk_mode<false>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w, sm.thr, sm.rab_ts_half);
         tmem_st16(s_tmem + ch * 16, pk);
       }
       tmem_wait_st();
@@ -501,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t orr[32];
         if (cnt > 0) {
           tmem_ld32(tmem + lane_base + 256 + x * 128 + ch * 32, orr);
-          tmem_wait_ld();
+          tmem_wait_ld(orr);
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) orr[e] = 0u;
