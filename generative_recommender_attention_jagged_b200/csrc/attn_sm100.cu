@@ -28,7 +28,8 @@
 // it also stages the keys' timestamps and a window of 0.5*rab_pos in shared
 // memory), warp 9 MMA issuer and TMEM owner.  Tensor memory holds S_A, S_B,
 // O_A, O_B (4 x 128 columns); while one warpgroup turns S into P the tensor
-// core runs the other tile's GEMMs.  Every wait is bounded (about 2 s), after
+// core runs the other tile's GEMMs, and each 64-key half of P goes to the
+// A.V GEMM as soon as it is written.  Every wait is bounded (about 2 s), after
 // which the kernel reports HSTU_ERR_TIMEOUT and winds down.
 //
 // Elementwise work per score: hb = s/2 = (alpha/2) S + 0.5 (rab_pos + rab_ts)
@@ -40,7 +41,8 @@
 // compare tells whether a row stays in its bucket; a chunk where every row of
 // the warp does uses a constant, a chunk with at most one edge per row finds
 // it by a 5-step search and selects, and only chunks with more edges (next to
-// the diagonal) walk column by column.  The SiLU loop itself is branch-free.
+// the diagonal) take each column's bucket from an octave table (the bit length
+// of |dt| + 1 picks four integer edges).  The SiLU loop itself is branch-free.
 // The producer loads each tile's metadata into registers one tile ahead, so
 // its global-load latency hides behind the wait for a free stage.
 #include <cuda_bf16.h>
@@ -76,13 +78,15 @@ struct __align__(1024) Smem {
   Meta meta[kStages];
   long long thr[kMaxBuckets];
   float rab_ts_half[kMaxBuckets];
+  uint4 oct[32];
   uint64_t bar_q;
   uint64_t bar_k_full[kStages];
   uint64_t bar_v_full[kStages];
   uint64_t bar_meta_full[kStages];
   uint64_t bar_kv_empty[kStages];
   uint64_t bar_s_full[kQTiles];
-  uint64_t bar_p_full[kQTiles];
+  uint64_t bar_p_lo[kQTiles];  // P of keys 0-63 written
+  uint64_t bar_p_hi[kQTiles];  // P of keys 64-127 written
   uint64_t bar_o_full;
   uint32_t tmem_base;
   int abort;
@@ -161,19 +165,34 @@ __device__ __forceinline__ void walk_to(Walk& w, long long tj, const long long* 
 }
 
 // Time-bias modes of a 32-column chunk.
-enum BiasMode { kBiasConst = 0, kBiasEdge = 1, kBiasWalk = 2 };
+enum BiasMode { kBiasConst = 0, kBiasEdge = 1, kBiasOct = 2, kBiasWalk = 3 };
 
 // 32 scores of one row: S (fp32 bits) -> P (bf16 pairs).
 //   kBiasConst: the row's time bucket is the same over the chunk (w.tsb)
 //   kBiasEdge:  one bucket edge: columns before `pos` use tsb_lo, the rest w.tsb
-//   kBiasWalk:  per-column walk over the bucket edges
+//   kBiasOct:   every column's bucket from the octave table (|dt| + 1 < 2^32)
+//   kBiasWalk:  per-column walk over the bucket edges (wider gaps)
 // MASK zeroes the columns past climit.
 template <int MODE, bool MASK>
 __device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&pk)[16], const float* wp,
                                            const long long* ts, int col0, int climit, int pos, float tsb_lo,
-                                           float alpha_half, Walk& w, const long long* thr, const float* rts) {
+                                           float alpha_half, Walk& w, const long long* thr, const float* rts,
+                                           const uint4* oct) {
   float tsv[32];
-  if constexpr (MODE == kBiasWalk) {
+  if constexpr (MODE == kBiasOct) {
+    const unsigned int ti1 = (unsigned int)(w.t_i + 1);  // low words: the differences fit in 32 bits
+    int b = 0;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      unsigned int x = ti1 - (unsigned int)ts[col0 + c];
+      x = max(x, 1u);  // keys later than the row exist only in masked columns
+      b = bucket_oct(oct, x);
+      tsv[c] = rts[b];
+    }
+    w.b = b;
+    w.tlim = w.t_i + 1 - thr[b];
+    w.tsb = rts[b];
+  } else if constexpr (MODE == kBiasWalk) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
       walk_to(w, ts[col0 + c], thr, rts);
@@ -212,13 +231,15 @@ template <bool MASK>
 __device__ __forceinline__ void silu_chunk_mode(int mode, const uint32_t (&sr)[32], uint32_t (&pk)[16],
                                                 const float* wp, const long long* ts, int col0, int climit,
                                                 int pos, float tsb_lo, float alpha_half, Walk& w,
-                                                const long long* thr, const float* rts) {
+                                                const long long* thr, const float* rts, const uint4* oct) {
   if (mode == kBiasConst)
-    silu_chunk<kBiasConst, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts);
+    silu_chunk<kBiasConst, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
   else if (mode == kBiasEdge)
-    silu_chunk<kBiasEdge, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts);
+    silu_chunk<kBiasEdge, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+  else if (mode == kBiasOct)
+    silu_chunk<kBiasOct, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
   else
-    silu_chunk<kBiasWalk, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts);
+    silu_chunk<kBiasWalk, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -261,7 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < kQTiles; ++x) {
       mbar_init(&sm.bar_s_full[x], 1);
-      mbar_init(&sm.bar_p_full[x], kTile);
+      mbar_init(&sm.bar_p_lo[x], kTile);
+      mbar_init(&sm.bar_p_hi[x], kTile);
     }
     mbar_init(&sm.bar_o_full, 1);
     sm.abort = 0;
@@ -271,6 +293,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.thr[x] = tab.thr[x];
     sm.rab_ts_half[x] = x < a.nb ? 0.5f * a.rab_ts[x] : 0.f;
   }
+  if (threadIdx.x < 32)
+    sm.oct[threadIdx.x] = make_uint4(tab.oct[threadIdx.x][0], tab.oct[threadIdx.x][1], tab.oct[threadIdx.x][2],
+                                     tab.oct[threadIdx.x][3]);
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -437,10 +462,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&sm.bar_s_full[x]);
       };
-      auto issue_pv = [&](int x, int t) {
+      // O_X += P_X V over keys [64 h, 64 h + 64): P columns 32 h.., V rows 64 h..
+      auto issue_pv_half = [&](int x, int t, int h) {
         const uint32_t v_base = smem_u32(sm.v[t % kStages]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
           mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, sw128_desc(v_base + kk * 2048, kHalfBytes, 1024),
                  idesc_pv, (t > 0 || kk > 0));
       };
@@ -456,11 +482,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool v_ready = false, k_next_ready = false;
         for (int x = 0; ok && x < kQTiles; ++x) {
           if (t >= cnt[x]) continue;
-          ok = mbar_wait(&sm.bar_p_full[x], t & 1, abort_flag, a.hdr, 4);
+          ok = mbar_wait(&sm.bar_p_lo[x], t & 1, abort_flag, a.hdr, 4);
           if (ok && !v_ready) ok = v_ready = mbar_wait(&sm.bar_v_full[s], (t / kStages) & 1, abort_flag, a.hdr, 5);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(x, t);
+          issue_pv_half(x, t, 0);
+          ok = mbar_wait(&sm.bar_p_hi[x], t & 1, abort_flag, a.hdr, 4);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv_half(x, t, 1);
           if (t + 1 < cnt[x]) {
             if (!k_next_ready)
               ok = k_next_ready = mbar_wait(&sm.bar_k_full[(t + 1) % kStages], ((t + 1) / kStages) & 1,
@@ -534,6 +564,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(~0u, uni)) {
           const long long tlim2 = w.b > 0 ? w.t_i + 1 - sm.thr[w.b - 1] : LLONG_MIN;
           const bool one = uni || t_last <= tlim2;              // at most one edge in the chunk
+          // octave mode needs |dt| + 1 < 2^32 at the chunk's first allowed column
+          const bool narrow = uni || (w.t_i + 1 - m.ts[col0]) < (1ll << 32);
           if (__all_sync(~0u, one)) {
             mode = kBiasEdge;
             if (!uni) {
@@ -547,20 +579,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               w.tsb = sm.rab_ts_half[w.b];
             }
           } else {
-            mode = kBiasWalk;
+            mode = __all_sync(~0u, narrow) ? kBiasOct : kBiasWalk;
           }
         }
         tmem_wait_ld(sr);
         uint32_t pk[16];
         if (need_mask)
-          silu_chunk_mode<true>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w, sm.thr, sm.rab_ts_half);
+          silu_chunk_mode<true>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w, sm.thr,
+                                sm.rab_ts_half, sm.oct);
         else
-          silu_chunk_mode<false>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w, sm.thr, sm.rab_ts_half);
+          silu_chunk_mode<false>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w, sm.thr,
+                                 sm.rab_ts_half, sm.oct);
         tmem_st16(s_tmem + ch * 16, pk);
+        if (ch & 1) {  // hand each 64-key half of P to the MMA as soon as it is written
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(ch == 1 ? &sm.bar_p_lo[x] : &sm.bar_p_hi[x]);
+        }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sm.bar_p_full[x]);
     }
     if (ok && cT > 0) {
       ok = ew_all(mbar_wait(&sm.bar_o_full, 0, abort_flag, a.hdr, 7), x);

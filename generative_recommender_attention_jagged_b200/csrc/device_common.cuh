@@ -40,6 +40,14 @@ __device__ __forceinline__ unsigned long long abs_dt_plus1(long long dt) {
   return m == ~0ull ? m : m + 1;
 }
 
+// bucket of a 32-bit x >= 1 from the octave table (see BucketTable::oct)
+__device__ __forceinline__ int bucket_oct(const uint4* oct, unsigned int x) {
+  unsigned int e;
+  asm("bfind.u32 %0, %1;" : "=r"(e) : "r"(x));
+  const uint4 t = oct[e];
+  return (int)t.x + (x >= t.y) + (x >= t.z) + (x >= t.w);
+}
+
 __device__ __forceinline__ int bucket_of_dt(const long long* thr, long long dt) {
   unsigned long long x = abs_dt_plus1(dt);
   // thresholds are < 2^63, so any x >= 2^63 lies above every finite edge

@@ -19,6 +19,10 @@ constexpr int kMaxSplits = 64;
 // largest b with thr[b] <= x, x = |dt| + 1.
 struct BucketTable {
   long long thr[kMaxBuckets];
+  // For x in [2^e, 2^(e+1)), e = 0..31: bucket(x) = oct[e][0] + #{k = 1..3 : x >= oct[e][k]}
+  // (an octave spans ln2/0.301 = 2.3 buckets, so it holds at most 3 edges);
+  // edges that are not reached are 0xFFFFFFFF.
+  unsigned int oct[32][4];
 };
 
 // Built once per process in exact binary128 arithmetic (ts_table.cpp).

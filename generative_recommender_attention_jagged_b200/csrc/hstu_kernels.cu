@@ -350,10 +350,16 @@ __global__ void __launch_bounds__(256) epilogue_kernel(const AttnArgs a) {
 __global__ void __launch_bounds__(256) ts_bucket_kernel(const int64_t* __restrict__ dt, int64_t n,
                                                         int32_t* __restrict__ out, const BucketTable tab) {
   __shared__ long long thr[kMaxBuckets];
+  __shared__ uint4 oct[32];
   for (int x = threadIdx.x; x < kMaxBuckets; x += blockDim.x) thr[x] = tab.thr[x];
+  for (int x = threadIdx.x; x < 32; x += blockDim.x)
+    oct[x] = make_uint4(tab.oct[x][0], tab.oct[x][1], tab.oct[x][2], tab.oct[x][3]);
   __syncthreads();
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-    out[i] = bucket_of_dt(thr, dt[i]);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const unsigned long long x = abs_dt_plus1(dt[i]);
+    // values below 2^32 take the octave table, larger ones the binary search
+    out[i] = x < (1ull << 32) ? bucket_oct(oct, (unsigned int)x) : bucket_of_dt(thr, dt[i]);
+  }
 }
 
 int num_sms() {

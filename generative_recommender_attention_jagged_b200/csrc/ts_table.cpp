@@ -43,6 +43,18 @@ const BucketTable& bucket_table(int num_buckets) {
   std::call_once(g_once[num_buckets], [num_buckets] {
     BucketTable& t = g_tables[num_buckets];
     for (int b = 0; b < kMaxBuckets; ++b) t.thr[b] = b < num_buckets ? edge_for(b) : LLONG_MAX;
+    // octave table: the bucket of 2^e and the (at most three) edges inside [2^e, 2^(e+1))
+    for (int e = 0; e < 32; ++e) {
+      const long long lo = 1ll << e, hi = (2ll << e) - 1;
+      int b_lo = 0;
+      for (int b = 0; b < kMaxBuckets; ++b)
+        if (t.thr[b] <= lo) b_lo = b;
+      t.oct[e][0] = (unsigned int)b_lo;
+      for (int k = 1; k <= 3; ++k) {
+        const int b = b_lo + k;
+        t.oct[e][k] = (b < kMaxBuckets && t.thr[b] <= hi) ? (unsigned int)t.thr[b] : 0xFFFFFFFFu;
+      }
+    }
   });
   return g_tables[num_buckets];
 }
