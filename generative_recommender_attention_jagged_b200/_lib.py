@@ -24,6 +24,7 @@ DT_BF16 = 1
 
 F_FORCE_SIMT = 0x1
 F_OUTPUT_RAW_AV = 0x2
+F_PRECISE_SILU = 0x4
 F_STAGE_PLAN = 0x10
 F_STAGE_ATTN = 0x20
 F_STAGE_EPILOGUE = 0x40

@@ -72,7 +72,7 @@ def hstu_attn_fwd(q, k, v, u, seq_offsets, timestamps, rab_pos, rab_ts, *, n_max
                   alpha: Optional[float] = None, num_candidates=None, ln_gamma=None, ln_beta=None,
                   ln_eps: float = 1e-5, max_seq_len: Optional[int] = None, out=None,
                   workspace=None, raw_av: bool = False, force_simt: bool = False, stages: int = 0,
-                  stream=None, params: Optional[_lib.AttnParams] = None):
+                  stream=None, params: Optional[_lib.AttnParams] = None, precise_silu: bool = False):
     """Jagged HSTU attention forward; returns out [T, H*d] (or o [T,H,d] fp32 when raw_av)."""
     T, H, d = q.shape
     dt = q.dtype
@@ -88,7 +88,8 @@ def hstu_attn_fwd(q, k, v, u, seq_offsets, timestamps, rab_pos, rab_ts, *, n_max
         raise ValueError("q, k and v must share one token stride")
     us = _rows_view("u", u, H, d)
     B = seq_offsets.numel() - 1
-    flags = (_lib.F_OUTPUT_RAW_AV if raw_av else 0) | (_lib.F_FORCE_SIMT if force_simt else 0) | stages
+    flags = ((_lib.F_OUTPUT_RAW_AV if raw_av else 0) | (_lib.F_FORCE_SIMT if force_simt else 0) |
+             (_lib.F_PRECISE_SILU if precise_silu else 0) | stages)
     if params is None:
         params = attn_params(batch=B, num_heads=H, head_dim=d, n_max=n_max, total_tokens=T,
                              max_seq_len=n_max if max_seq_len is None else max_seq_len, dtype=dt,
@@ -112,7 +113,8 @@ def hstu_attn_fwd_paged(q, k, v, u, new_offsets, timestamps, ts_offsets, rab_pos
                         num_candidates=None, ln_gamma=None, ln_beta=None, ln_eps: float = 1e-5,
                         max_seq_len: Optional[int] = None, num_splits: Optional[int] = None,
                         max_cached_len: Optional[int] = None, out=None, workspace=None,
-                        raw_av: bool = False, force_simt: bool = False, stages: int = 0, stream=None):
+                        raw_av: bool = False, force_simt: bool = False, stages: int = 0, stream=None,
+                        precise_silu: bool = False):
     """Incremental HSTU attention of new tokens over a paged K/V prefix."""
     T, H, d = q.shape
     dt = q.dtype
@@ -131,7 +133,8 @@ def hstu_attn_fwd_paged(q, k, v, u, new_offsets, timestamps, ts_offsets, rab_pos
         raise ValueError("q, k and v must share one token stride")
     us = _rows_view("u", u, H, d)
     B = new_offsets.numel() - 1
-    flags = (_lib.F_OUTPUT_RAW_AV if raw_av else 0) | (_lib.F_FORCE_SIMT if force_simt else 0) | stages
+    flags = ((_lib.F_OUTPUT_RAW_AV if raw_av else 0) | (_lib.F_FORCE_SIMT if force_simt else 0) |
+             (_lib.F_PRECISE_SILU if precise_silu else 0) | stages)
     params = attn_params(batch=B, num_heads=H, head_dim=d, n_max=n_max, total_tokens=T,
                          max_seq_len=n_max if max_seq_len is None else max_seq_len, dtype=dt,
                          alpha=alpha, num_ts_buckets=rab_ts.numel(), qkv_stride=qs, u_stride=us,

@@ -8,9 +8,9 @@
 //   S_X  = Q_X K^T          tcgen05.mma, A = Q_X (smem, K-major), B = K (smem,
 //                           K-major), fp32 accumulator in tensor memory
 //   P_X  = SiLU(alpha S_X + rab_pos[p_i - p_j + N - 1] + rab_ts[bucket(t_i - t_j)]),
-//          0 outside the allowed set; computed by the elementwise warpgroup of
-//          X, which reads S_X with tcgen05.ld and writes P_X as bf16 pairs back
-//          over S_X (tcgen05.st)
+//          0 outside the allowed set; computed by the two elementwise
+//          warpgroups of X (64 keys each), which read S_X with tcgen05.ld and
+//          write P_X as bf16 pairs back over their own half of S_X (tcgen05.st)
 //   O_X += P_X V            tcgen05.mma, A = P_X (tensor memory), B = V (smem, MN-major)
 //
 // There is no softmax, no row maximum and no rescaling: the weights are
@@ -22,18 +22,23 @@
 // the candidate's own term a_ii v_i is added by the epilogue, so no tile of
 // the candidate x candidate block is ever issued.
 //
-// Warp roles (320 threads): warps 0-3 elementwise for tile A, warps 4-7 for
-// tile B (thread = query row = TMEM lane), warp 8 producer (Q once; K/V
+// Warp roles (576 threads): warps 0-15 elementwise in four warpgroups, one
+// per (query tile, 64-key half of every key tile) (thread = query row = TMEM
+// lane; a warp reaches the lanes of its rank in the warpgroup), warp 16
+// producer (Q once; K/V
 // through a 2-stage ring by TMA, the paged prefix page by page; per key tile
 // it also stages the keys' timestamps and a window of 0.5*rab_pos in shared
-// memory), warp 9 MMA issuer and TMEM owner.  Tensor memory holds S_A, S_B,
+// memory), warp 17 MMA issuer and TMEM owner.  Tensor memory holds S_A, S_B,
 // O_A, O_B (4 x 128 columns); while one warpgroup turns S into P the tensor
 // core runs the other tile's GEMMs, and each 64-key half of P goes to the
 // A.V GEMM as soon as it is written.  Every wait is bounded (about 2 s), after
 // which the kernel reports HSTU_ERR_TIMEOUT and winds down.
 //
 // Elementwise work per score: hb = s/2 = (alpha/2) S + 0.5 (rab_pos + rab_ts)
-// with packed f32x2 FMA, SiLU(s) = hb (1 + tanh hb) with one MUFU tanh.  Time
+// with packed f32x2 FMA, then SiLU(s) = hb (1 + tanh hb): by default hb is
+// rounded to bf16 and one packed bf16x2 tanh and one bf16x2 FMA produce two
+// scores of P at once (P is bf16 for the A.V GEMM anyway); with the precise
+// option tanh and the FMA run in fp32 and P is rounded once.  Time
 // buckets are exact: a thread finds the bucket of its row's first key once per
 // work item by a binary search over integer edges, then walks down the edges
 // as the keys come closer in time (timestamps are non-decreasing inside a
@@ -55,9 +60,10 @@ namespace hstu {
 namespace {
 
 constexpr int kQTiles = 2;
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kEwWarps = 16;                 // 4 warpgroups: (query tile, 64-column half)
+constexpr int kThreads = 32 * (kEwWarps + 2);
+constexpr int kProducerWarp = kEwWarps;
+constexpr int kMmaWarp = kEwWarps + 1;
 constexpr int kStages = 2;
 constexpr int kTileBytes = kTile * 128 * 2;  // 128 rows x 128 bf16 = 32 KB
 constexpr int kHalfBytes = kTile * 128;      // 128 rows x 64 bf16: one 128B-swizzled box
@@ -116,7 +122,7 @@ __device__ __forceinline__ float4 lds_f4(const float* p) {
   return r;
 }
 
-// the 128 threads of one elementwise warpgroup agree on a flag
+// the 128 threads of one elementwise warpgroup (0..3) agree on a flag
 __device__ __forceinline__ bool ew_all(bool ok, int group) {
   uint32_t r;
   asm volatile(
@@ -173,37 +179,28 @@ enum BiasMode { kBiasConst = 0, kBiasEdge = 1, kBiasOct = 2, kBiasWalk = 3 };
 //   kBiasOct:   every column's bucket from the octave table (|dt| + 1 < 2^32)
 //   kBiasWalk:  per-column walk over the bucket edges (wider gaps)
 // MASK zeroes the columns past climit.
-template <int MODE, bool MASK>
+template <int MODE, bool MASK, bool PRECISE>
 __device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&pk)[16], const float* wp,
                                            const long long* ts, int col0, int climit, int pos, float tsb_lo,
                                            float alpha_half, Walk& w, const long long* thr, const float* rts,
                                            const uint4* oct) {
-  float tsv[32];
-  if constexpr (MODE == kBiasOct) {
-    const unsigned int ti1 = (unsigned int)(w.t_i + 1);  // low words: the differences fit in 32 bits
-    int b = 0;
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      unsigned int x = ti1 - (unsigned int)ts[col0 + c];
-      x = max(x, 1u);  // keys later than the row exist only in masked columns
-      b = bucket_oct(oct, x);
-      tsv[c] = rts[b];
-    }
-    w.b = b;
-    w.tlim = w.t_i + 1 - thr[b];
-    w.tsb = rts[b];
-  } else if constexpr (MODE == kBiasWalk) {
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      walk_to(w, ts[col0 + c], thr, rts);
-      tsv[c] = w.tsb;
-    }
-  } else if constexpr (MODE == kBiasEdge) {
-#pragma unroll
-    for (int c = 0; c < 32; ++c) tsv[c] = (col0 + c < pos) ? tsb_lo : w.tsb;
-  }
   const uint64_t ah2 = pk2(alpha_half, alpha_half);
   const uint64_t tsb2 = pk2(w.tsb, w.tsb);
+  const unsigned int ti1 = (unsigned int)(w.t_i + 1);  // octave mode: differences fit in 32 bits
+  int b_last = 0;
+  // time bias of column col (0.5 * rab_ts[bucket]) in the chunk's mode
+  auto ts_bias = [&](int col) -> float {
+    if constexpr (MODE == kBiasEdge) {
+      return col < pos ? tsb_lo : w.tsb;
+    } else if constexpr (MODE == kBiasOct) {
+      const unsigned int x = max(ti1 - (unsigned int)ts[col], 1u);  // later keys only in masked columns
+      b_last = bucket_oct(oct, x);
+      return rts[b_last];
+    } else {
+      walk_to(w, ts[col], thr, rts);
+      return w.tsb;
+    }
+  };
 #pragma unroll
   for (int c4 = 0; c4 < 8; ++c4) {
     const float4 w4 = lds_f4(wp + col0 + 4 * c4);
@@ -211,37 +208,56 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&
     for (int hlf = 0; hlf < 2; ++hlf) {
       const int c = 4 * c4 + 2 * hlf;
       uint64_t bias2 = hlf == 0 ? pk2(w4.x, w4.y) : pk2(w4.z, w4.w);
-      bias2 = add2(bias2, MODE == kBiasConst ? tsb2 : pk2(tsv[c], tsv[c + 1]));
+      if constexpr (MODE == kBiasConst) {
+        bias2 = add2(bias2, tsb2);
+      } else {
+        const float t0 = ts_bias(col0 + c);
+        const float t1 = ts_bias(col0 + c + 1);
+        bias2 = add2(bias2, pk2(t0, t1));
+      }
       const uint64_t h2 = fma2(pk2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), ah2, bias2);
       float h0, h1;
       upk2(h2, h0, h1);
-      const uint64_t p2 = fma2(h2, pk2(tanh_approx(h0), tanh_approx(h1)), h2);  // hb (1 + tanh hb)
-      float p0, p1;
-      upk2(p2, p0, p1);
-      if constexpr (MASK) {
-        p0 = (col0 + c <= climit) ? p0 : 0.f;
-        p1 = (col0 + c + 1 <= climit) ? p1 : 0.f;
+      if constexpr (MASK) {  // SiLU(0) = 0 exactly: masking hb masks P
+        h0 = (col0 + c <= climit) ? h0 : 0.f;
+        h1 = (col0 + c + 1 <= climit) ? h1 : 0.f;
       }
-      pk[c >> 1] = pack_bf16x2(p0, p1);
+      if constexpr (PRECISE) {
+        // fp32: P = hb (1 + tanh hb), one MUFU tanh per score, rounded once to bf16
+        const uint64_t p2 = fma2(pk2(h0, h1), pk2(tanh_approx(h0), tanh_approx(h1)), pk2(h0, h1));
+        float p0, p1;
+        upk2(p2, p0, p1);
+        pk[c >> 1] = pack_bf16x2(p0, p1);
+      } else {
+        // packed bf16: one MUFU tanh per two scores; P = hb (1 + tanh hb) as one bf16x2 FMA
+        const uint32_t hb = pack_bf16x2(h0, h1);
+        pk[c >> 1] = fma_bf16x2(hb, tanh_bf16x2(hb), hb);
+      }
     }
+  }
+  if constexpr (MODE == kBiasOct) {  // the walk state continues from the chunk's last column
+    w.b = b_last;
+    w.tlim = w.t_i + 1 - thr[b_last];
+    w.tsb = rts[b_last];
   }
 }
 
-template <bool MASK>
+template <bool MASK, bool PRECISE>
 __device__ __forceinline__ void silu_chunk_mode(int mode, const uint32_t (&sr)[32], uint32_t (&pk)[16],
                                                 const float* wp, const long long* ts, int col0, int climit,
                                                 int pos, float tsb_lo, float alpha_half, Walk& w,
                                                 const long long* thr, const float* rts, const uint4* oct) {
   if (mode == kBiasConst)
-    silu_chunk<kBiasConst, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+    silu_chunk<kBiasConst, MASK, PRECISE>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
   else if (mode == kBiasEdge)
-    silu_chunk<kBiasEdge, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+    silu_chunk<kBiasEdge, MASK, PRECISE>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
   else if (mode == kBiasOct)
-    silu_chunk<kBiasOct, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+    silu_chunk<kBiasOct, MASK, PRECISE>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
   else
-    silu_chunk<kBiasWalk, MASK>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+    silu_chunk<kBiasWalk, MASK, PRECISE>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
 }
 
+template <bool PRECISE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const AttnArgs a, const BucketTable tab, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -462,13 +478,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&sm.bar_s_full[x]);
       };
-      // O_X += P_X V over keys [64 h, 64 h + 64): P columns 32 h.., V rows 64 h..
+      // O_X += P_X V over keys [64 h, 64 h + 64): P at columns 64 h .. 64 h + 31 of
+      // S_X (16 keys per 8 columns), V rows 64 h..
       auto issue_pv_half = [&](int x, int t, int h) {
         const uint32_t v_base = smem_u32(sm.v[t % kStages]);
 #pragma unroll
         for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-          mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, sw128_desc(v_base + kk * 2048, kHalfBytes, 1024),
-                 idesc_pv, (t > 0 || kk > 0));
+          mma_ts(tmem + 256 + x * 128, tmem + x * 128 + 64 * h + (kk - 4 * h) * 8,
+                 sw128_desc(v_base + kk * 2048, kHalfBytes, 1024), idesc_pv, (t > 0 || kk > 0));
       };
       bool ok = cT == 0 || mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 2);
       if (ok && cT > 0) ok = mbar_wait(&sm.bar_k_full[0], 0, abort_flag, a.hdr, 3);
@@ -509,7 +526,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ elementwise
-    const int x = warp >> 2;                 // query tile of this warpgroup
+    const int x = warp >> 3;                 // query tile of this warpgroup
+    const int half = (warp >> 2) & 1;        // key columns 64*half .. 64*half + 63 of every tile
+    const int group = warp >> 2;             // warpgroup index 0..3
     const int r = threadIdx.x & (kTile - 1); // query row of the tile == TMEM lane
     const TileGeom& g = x == 0 ? gA : gB;
     const int cnt = x == 0 ? cA : cB;
@@ -536,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       key_tile(g, tb + t, k0, width);
       ok = mbar_wait(&sm.bar_meta_full[s], (t / kStages) & 1, abort_flag, a.hdr, 6);
       ok = ok && mbar_wait(&sm.bar_s_full[x], t & 1, abort_flag, a.hdr, 6);
-      ok = ew_all(ok, x);
+      ok = ew_all(ok, group);
       if (!ok) break;
       tc_fence_after();
       const Meta& m = sm.meta[s];
@@ -549,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool need_mask = !__all_sync(~0u, climit >= kTile - 1);
       const float* wp = &m.win[wcopy][woff];
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
         uint32_t sr[32];
         tmem_ld32(s_tmem + ch * 32, sr);
         // time-bias mode of this chunk (decided while the TMEM load is in flight):
@@ -585,27 +604,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld(sr);
         uint32_t pk[16];
         if (need_mask)
-          silu_chunk_mode<true>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w, sm.thr,
-                                sm.rab_ts_half, sm.oct);
+          silu_chunk_mode<true, PRECISE>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w,
+                                         sm.thr, sm.rab_ts_half, sm.oct);
         else
-          silu_chunk_mode<false>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w, sm.thr,
-                                 sm.rab_ts_half, sm.oct);
-        tmem_st16(s_tmem + ch * 16, pk);
-        if (ch & 1) {  // hand each 64-key half of P to the MMA as soon as it is written
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(ch == 1 ? &sm.bar_p_lo[x] : &sm.bar_p_hi[x]);
-        }
+          silu_chunk_mode<false, PRECISE>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w,
+                                          sm.thr, sm.rab_ts_half, sm.oct);
+        // P of this chunk packs into the warpgroup's own (already read) S columns:
+        // keys 0-63 at columns 0-31, keys 64-127 at columns 64-95
+        tmem_st16(s_tmem + half * 64 + (ch & 1) * 16, pk);
       }
+      // this warpgroup's 64-key half of P goes to the A.V GEMM
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(half == 0 ? &sm.bar_p_lo[x] : &sm.bar_p_hi[x]);
     }
     if (ok && cT > 0) {
-      ok = ew_all(mbar_wait(&sm.bar_o_full, 0, abort_flag, a.hdr, 7), x);
+      ok = ew_all(mbar_wait(&sm.bar_o_full, 0, abort_flag, a.hdr, 7), group);
       tc_fence_after();
     }
     if (ok && exists) {
       float* orow = a.o_ws + (((size_t)it.split * a.T_q + (g.qrow0 + r)) * a.H + it.head) * kHeadDim;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
         uint32_t orr[32];
         if (cnt > 0) {
           tmem_ld32(tmem + lane_base + 256 + x * 128 + ch * 32, orr);
@@ -640,13 +660,19 @@ cudaError_t launch_attn_sm100(const AttnArgs& a, const BucketTable& thr, const C
   cudaGetDevice(&dev);
   static unsigned long long attr_set = 0;  // one bit per device
   if (dev < 64 && !(attr_set & (1ull << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set |= 1ull << dev;
   }
   if (a.max_items <= 0) return cudaSuccess;
-  attn_sm100_kernel<<<a.max_items, kThreads, kSmemBytes, s>>>(a, thr, tm_q, tm_k, tm_v, tm_kpool, tm_vpool);
+  if (a.precise_silu)
+    attn_sm100_kernel<true><<<a.max_items, kThreads, kSmemBytes, s>>>(a, thr, tm_q, tm_k, tm_v, tm_kpool, tm_vpool);
+  else
+    attn_sm100_kernel<false><<<a.max_items, kThreads, kSmemBytes, s>>>(a, thr, tm_q, tm_k, tm_v, tm_kpool, tm_vpool);
   return cudaGetLastError();
 }
 

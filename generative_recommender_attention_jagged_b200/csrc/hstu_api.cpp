@@ -89,8 +89,8 @@ int check_params(const hstu_attn_params* p) {
     return HSTU_ERR_INVALID_ARG;
   if (p->num_ts_buckets <= 0 || p->num_ts_buckets > kMaxBuckets) return HSTU_ERR_UNSUPPORTED;
   if (p->dtype != HSTU_DT_F32 && p->dtype != HSTU_DT_BF16) return HSTU_ERR_INVALID_ARG;
-  const uint32_t known = HSTU_F_FORCE_SIMT | HSTU_F_OUTPUT_RAW_AV | HSTU_F_STAGE_PLAN | HSTU_F_STAGE_ATTN |
-                         HSTU_F_STAGE_EPILOGUE;
+  const uint32_t known = HSTU_F_FORCE_SIMT | HSTU_F_OUTPUT_RAW_AV | HSTU_F_PRECISE_SILU | HSTU_F_STAGE_PLAN |
+                         HSTU_F_STAGE_ATTN | HSTU_F_STAGE_EPILOGUE;
   if (p->flags & ~known) return HSTU_ERR_INVALID_ARG;
   if (p->head_dim > 256 || (long long)p->num_heads * p->head_dim > 1024) return HSTU_ERR_UNSUPPORTED;
   const int qs = p->qkv_stride ? p->qkv_stride : p->num_heads * p->head_dim;
@@ -150,7 +150,7 @@ int run(const hstu_attn_params* p, const Common& c) {
                   c.num_pages <= 0 || c.max_pages <= 0))
     return HSTU_ERR_INVALID_ARG;
   if (c.splits < 1 || c.splits > kMaxSplits) return HSTU_ERR_INVALID_ARG;
-  const void* ptrs[] = {c.q, c.k, c.v, c.u, c.out, c.ws, c.k_pool, c.v_pool};
+  const void* ptrs[] = {c.q, c.k, c.v, c.u, c.out, c.ws, c.k_pool, c.v_pool, c.gamma, c.beta};
   for (const void* ptr : ptrs)
     if (ptr && !aligned16(ptr)) return HSTU_ERR_ALIGNMENT;
   const bool tc = use_tensor_cores(p);
@@ -184,6 +184,7 @@ int run(const hstu_attn_params* p, const Common& c) {
   a.self_term = tc ? 1 : 0;
   a.out_bf16 = p->dtype == HSTU_DT_BF16 ? 1 : 0;
   a.in_bf16 = p->dtype == HSTU_DT_BF16 ? 1 : 0;
+  a.precise_silu = (p->flags & HSTU_F_PRECISE_SILU) ? 1 : 0;
   a.q = c.q;
   a.k = c.k;
   a.v = c.v;

@@ -61,6 +61,7 @@ struct AttnArgs {
   int32_t self_term;    // epilogue adds a_ii v_i for candidate rows (tensor-core path)
   int32_t out_bf16;     // out dtype
   int32_t in_bf16;      // q/k/v/u/pool dtype
+  int32_t precise_silu; // tensor-core path: fp32 tanh per score instead of packed bf16x2
   const void* q;
   const void* k;
   const void* v;

@@ -344,6 +344,132 @@ __global__ void __launch_bounds__(256) epilogue_kernel(const AttnArgs a) {
   }
 }
 
+// Vectorised epilogue for D = H*d a multiple of 128 (D = 128 * VPT): lane l
+// holds features 128 k + 4 l .. 128 k + 4 l + 3 (float4 loads of the partial
+// sums, 8-byte loads/stores of bf16).  Same arithmetic as epilogue_kernel.
+template <int VPT, typename TIn, typename TOut>
+__global__ void __launch_bounds__(256) epilogue_vec_kernel(const AttnArgs a) {
+  if (a.hdr->status != 0) return;
+  const int lane = threadIdx.x & 31;
+  const int warps_per_block = blockDim.x >> 5;
+  constexpr int D = 128 * VPT;
+  const float inv_n = 1.0f / (float)a.n_max;
+  const size_t split_stride = (size_t)a.T_q * D;
+  for (int row = blockIdx.x * warps_per_block + (threadIdx.x >> 5); row < a.T_q;
+       row += gridDim.x * warps_per_block) {
+    float o[VPT][4];
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const float4* src = reinterpret_cast<const float4*>(a.o_ws + (size_t)row * D + 128 * k + 4 * lane);
+      float4 acc = src[0];
+      for (int sp = 1; sp < a.num_splits; ++sp) {
+        const float4 v = src[sp * split_stride / 4];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      o[k][0] = acc.x;
+      o[k][1] = acc.y;
+      o[k][2] = acc.z;
+      o[k][3] = acc.w;
+    }
+    if (a.self_term && a.num_cand) {
+      const int u = find_user(a.q_offsets, a.B, row);
+      const int q0 = a.q_offsets[u];
+      const int nq = a.q_offsets[u + 1] - q0;
+      if (row - q0 >= nq - a.num_cand[u]) {
+        const float bias = a.rab_pos[a.n_max - 1] + a.rab_ts[0];
+        const TIn* q = static_cast<const TIn*>(a.q) + (size_t)row * a.qkv_stride;
+        const TIn* kk = static_cast<const TIn*>(a.k) + (size_t)row * a.qkv_stride;
+        const TIn* v = static_cast<const TIn*>(a.v) + (size_t)row * a.qkv_stride;
+        // head h covers features [h d, (h+1) d); d is a multiple of 4 here
+        for (int h = 0; h < a.H; ++h) {
+          float part = 0.f;
+#pragma unroll
+          for (int k = 0; k < VPT; ++k)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int e = 128 * k + 4 * lane + c;
+              if (e / a.d == h) part = fmaf(to_f(q[e]), to_f(kk[e]), part);
+            }
+          const float sc = a.alpha * warp_sum(part) + bias;
+          const float wgt = sc / (1.f + expf(-sc));
+#pragma unroll
+          for (int k = 0; k < VPT; ++k)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int e = 128 * k + 4 * lane + c;
+              if (e / a.d == h) o[k][c] = fmaf(wgt, to_f(v[e]), o[k][c]);
+            }
+        }
+      }
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        o[k][c] *= inv_n;
+        sum += o[k][c];
+      }
+    if (a.out_raw) {
+#pragma unroll
+      for (int k = 0; k < VPT; ++k)
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + (size_t)row * D + 128 * k + 4 * lane) =
+            make_float4(o[k][0], o[k][1], o[k][2], o[k][3]);
+      continue;
+    }
+    const float mean = warp_sum(sum) / (float)D;
+    float sq = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float cc = o[k][c] - mean;
+        sq = fmaf(cc, cc, sq);
+      }
+    const float rstd = rsqrtf(warp_sum(sq) / (float)D + a.ln_eps);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int e0 = 128 * k + 4 * lane;
+      float g[4] = {1.f, 1.f, 1.f, 1.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
+      if (a.ln_gamma) {
+        const float4 gg = *reinterpret_cast<const float4*>(a.ln_gamma + e0);
+        g[0] = gg.x; g[1] = gg.y; g[2] = gg.z; g[3] = gg.w;
+      }
+      if (a.ln_beta) {
+        const float4 bb = *reinterpret_cast<const float4*>(a.ln_beta + e0);
+        b[0] = bb.x; b[1] = bb.y; b[2] = bb.z; b[3] = bb.w;
+      }
+      float uv[4], y[4];
+      const TIn* up = static_cast<const TIn*>(a.u) + (size_t)row * a.u_stride + e0;
+      if constexpr (sizeof(TIn) == 2) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(up);
+        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+        uv[0] = __low2float(lo); uv[1] = __high2float(lo); uv[2] = __low2float(hi); uv[3] = __high2float(hi);
+      } else {
+        const float4 f = *reinterpret_cast<const float4*>(up);
+        uv[0] = f.x; uv[1] = f.y; uv[2] = f.z; uv[3] = f.w;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) y[c] = ((o[k][c] - mean) * rstd * g[c] + b[c]) * uv[c];
+      TOut* out = static_cast<TOut*>(a.out) + (size_t)row * D + e0;
+      if constexpr (sizeof(TOut) == 2) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(y[0], y[1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(y[2], y[3]);
+        uint2 raw;
+        raw.x = *reinterpret_cast<uint32_t*>(&lo);
+        raw.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(out) = raw;
+      } else {
+        *reinterpret_cast<float4*>(out) = make_float4(y[0], y[1], y[2], y[3]);
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // standalone time-bucket kernel
 // ---------------------------------------------------------------------------
@@ -393,8 +519,31 @@ cudaError_t launch_attn_simt(const AttnArgs& a, const BucketTable& thr, cudaStre
   return cudaGetLastError();
 }
 
+template <typename TIn, typename TOut>
+bool launch_epilogue_vec(const AttnArgs& a, int blocks, cudaStream_t s) {
+  const int D = a.H * a.d;
+  if (D % 128 != 0 || a.d % 4 != 0) return false;
+  switch (D / 128) {
+    case 1: epilogue_vec_kernel<1, TIn, TOut><<<blocks, 256, 0, s>>>(a); return true;
+    case 2: epilogue_vec_kernel<2, TIn, TOut><<<blocks, 256, 0, s>>>(a); return true;
+    case 4: epilogue_vec_kernel<4, TIn, TOut><<<blocks, 256, 0, s>>>(a); return true;
+    case 8: epilogue_vec_kernel<8, TIn, TOut><<<blocks, 256, 0, s>>>(a); return true;
+    default: return false;
+  }
+}
+
 cudaError_t launch_epilogue(const AttnArgs& a, cudaStream_t s) {
   const int blocks = std::max(1, std::min((a.T_q + 7) / 8, num_sms() * 16));
+  // rows of u are 16-byte aligned (the host checks strides), so the
+  // vectorised kernel applies whenever H*d is a multiple of 128
+  {
+    bool done = false;
+    if (a.in_bf16) done = a.out_bf16 ? launch_epilogue_vec<__nv_bfloat16, __nv_bfloat16>(a, blocks, s)
+                                     : launch_epilogue_vec<__nv_bfloat16, float>(a, blocks, s);
+    else done = a.out_bf16 ? launch_epilogue_vec<float, __nv_bfloat16>(a, blocks, s)
+                           : launch_epilogue_vec<float, float>(a, blocks, s);
+    if (done) return cudaGetLastError();
+  }
   if (a.in_bf16) {
     if (a.out_bf16) epilogue_kernel<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, s>>>(a);
     else epilogue_kernel<__nv_bfloat16, float><<<blocks, 256, 0, s>>>(a);

@@ -41,7 +41,8 @@
  *     above n_max, unsorted timestamps, page ids out of range, a wait that ran
  *     out) are written to a status word inside the workspace and read with
  *     hstu_check_device_error().
- *   - Device pointers must be 16-byte aligned; q/k/v/u row strides must be
+ *   - Device pointers (including ln_gamma, ln_beta) must be 16-byte aligned;
+ *     q/k/v/u row strides must be
  *     multiples of 8 elements (bf16) or 4 elements (fp32).
  *   - `out` must not alias any input.
  *   - Within one user, timestamps must be non-decreasing (the pages' inputs
@@ -82,6 +83,8 @@ typedef enum { HSTU_DT_F32 = 0, HSTU_DT_BF16 = 1 } hstu_dtype;
 /* flags */
 #define HSTU_F_FORCE_SIMT     0x1u  /* use the CUDA-core kernel even where the tensor-core one applies */
 #define HSTU_F_OUTPUT_RAW_AV  0x2u  /* write o = A.V as fp32 [T,H,d] to `out` instead of y            */
+#define HSTU_F_PRECISE_SILU   0x4u  /* tensor-core path: SiLU with an fp32 tanh per score (slower);
+                                       default: packed bf16x2 tanh/FMA, P is bf16 either way         */
 #define HSTU_F_STAGE_PLAN     0x10u /* run only the validate + tile-schedule kernels                    */
 #define HSTU_F_STAGE_ATTN     0x20u /* run only the attention kernel (needs a plan in the workspace)    */
 #define HSTU_F_STAGE_EPILOGUE 0x40u /* run only the LayerNorm-gate epilogue (needs the attention part)  */

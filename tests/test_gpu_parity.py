@@ -339,3 +339,17 @@ def test_tensor_core_path_is_the_one_that_runs():
     o_simt = run_jagged(b, raw_av=True, force_simt=True).cpu()
     assert not torch.equal(o_tc, o_simt)
     assert rel_err(host64(o_tc), host64(o_simt)) <= BF16_TOL
+
+
+@pytest.mark.parametrize("precise", [False, True])
+def test_silu_paths_both_within_tolerance(precise):
+    # default: packed bf16x2 tanh/FMA; precise: fp32 tanh per score
+    b = small_batch([900, 400, 129], cands=[0, 100, 0], n_max=1024, seed=31)
+    rng = np.random.default_rng(4)
+    b.rab_pos = rng.normal(0, 0.5, size=2 * b.n_max - 1).astype(np.float32)
+    b.rab_ts = rng.normal(0, 0.5, size=128).astype(np.float32)
+    want_y, want_o = oracle.batch_attn(b, want_o=True)
+    o = host64(run_jagged(b, raw_av=True, precise_silu=precise))
+    y = host64(run_jagged(b, precise_silu=precise))
+    assert rel_err(o, want_o) <= BF16_TOL
+    assert rel_err(y, want_y) <= BF16_TOL
