@@ -178,3 +178,33 @@ def hstu_status_string(status: int) -> str:
 
 def hstu_version() -> int:
     return int(_lib.load().hstu_version())
+
+
+def hstu_attn_fwd_static_ws(q, k, v, u, seq_offsets, timestamps, rab_pos, rab_ts, *, n_max: int,
+                            alpha: Optional[float] = None, num_candidates=None, ln_gamma=None,
+                            ln_beta=None, ln_eps: float = 1e-5, max_seq_len: Optional[int] = None,
+                            out=None, stream=None):
+    """hstu_attn_fwd without a workspace: the library's own 16 MiB device scratch is
+    used instead (for callers that cannot allocate device memory where they run
+    attention).  `out` may be given so that the call allocates nothing at all."""
+    T, H, d = q.shape
+    dt = q.dtype
+    for name, t in (("q", q), ("k", k), ("v", v), ("u", u)):
+        _need_cuda(name, t, dt)
+    qs = _rows_view("q", q, H, d)
+    us = _rows_view("u", u, H, d)
+    params = attn_params(batch=seq_offsets.numel() - 1, num_heads=H, head_dim=d, n_max=n_max,
+                         total_tokens=T, max_seq_len=n_max if max_seq_len is None else max_seq_len,
+                         dtype=dt, alpha=alpha, num_ts_buckets=rab_ts.numel(), qkv_stride=qs,
+                         u_stride=us, ln_eps=ln_eps)
+    if out is None:
+        out = torch.empty(T, H * d, dtype=dt, device=q.device)
+    lib = _lib.load()
+    fn = lib.hstu_attn_fwd_static_ws
+    fn.argtypes = [ctypes.POINTER(_lib.AttnParams)] + [ctypes.c_void_p] * 13
+    fn.restype = ctypes.c_int
+    rc = fn(ctypes.byref(params), _p(q), _p(k), _p(v), _p(u), _p(seq_offsets), _p(timestamps),
+            _p(num_candidates), _p(rab_pos), _p(rab_ts), _p(ln_gamma), _p(ln_beta), _p(out),
+            _stream(stream))
+    _lib.check(rc, "hstu_attn_fwd_static_ws")
+    return out
