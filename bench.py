@@ -330,7 +330,7 @@ def run_ours(args, rank, world, device):
                      "launch_ms": round(attn_avg_ms, 4), "flops_per_launch": flops_layer,
                      "issued_tile_tflops": round(issued_tflops, 2),
                      "issued_frac": round(issued_tflops / peak, 4)},
-        "gpu_launches": args.steps * L * 4,
+        "gpu_launches": args.steps * L * 3,  # per layer: plan, attention, epilogue
         "clocks": clk,
         "e2e": e2e,
     }
@@ -449,6 +449,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-paged", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--paged-only", action="store_true",
+                    help="run only the paged incremental sub-benchmark (profiling captures)")
     ap.add_argument("--layers", type=int, default=None,
                     help="fewer layers (profiling captures only; the bench line uses all 8)")
     args = ap.parse_args()
@@ -471,6 +473,10 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
+    if args.paged_only:
+        if rank == 0:
+            print(json.dumps({"paged": run_paged_bench(args, device)}), flush=True)
+        return
     result, b0 = run_ours(args, rank, world, device)
     if rank == 0 and not args.no_paged and world == 1:
         result["paged"] = run_paged_bench(args, device)

@@ -210,8 +210,7 @@ int run(const hstu_attn_params* p, const Common& c) {
   cudaError_t e = cudaSuccess;
   if (stages & HSTU_F_STAGE_PLAN) {
     if ((e = cudaMemsetAsync(c.ws, 0, sizeof(WsHeader), c.stream)) != cudaSuccess) return HSTU_ERR_CUDA;
-    if ((e = launch_validate(a, c.stream)) != cudaSuccess) return HSTU_ERR_CUDA;
-    if (tc && (e = launch_schedule(a, c.stream)) != cudaSuccess) return HSTU_ERR_CUDA;
+    if ((e = launch_plan(a, tc, p->max_seq_len, c.stream)) != cudaSuccess) return HSTU_ERR_CUDA;
   }
   if (a.T_q == 0) return HSTU_OK;
   if (stages & HSTU_F_STAGE_ATTN) {

@@ -33,7 +33,8 @@ struct WsHeader {
   int32_t status;      // first device-detected error (hstu_status), 0 = OK
   int32_t detail;      // user index or item that raised it
   int32_t n_items;     // work items written by the scheduler
-  int32_t pad[61];
+  int32_t blocks_done; // plan kernel: validation blocks finished (the last one schedules)
+  int32_t pad[60];
 };
 static_assert(sizeof(WsHeader) == 256, "header size");
 
@@ -102,8 +103,9 @@ struct TileGeom {
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Launchers implemented in the .cu files.  All return a cudaError_t.
-cudaError_t launch_validate(const AttnArgs& a, cudaStream_t s);
-cudaError_t launch_schedule(const AttnArgs& a, cudaStream_t s);
+// Validation of offsets, lengths, page ids and timestamps; with `schedule`
+// the last block to finish also builds the tensor-core work list.
+cudaError_t launch_plan(const AttnArgs& a, bool schedule, int max_seq_len, cudaStream_t s);
 cudaError_t launch_attn_sm100(const AttnArgs& a, const BucketTable& thr, const CUtensorMap& tm_q,
                               const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                               const CUtensorMap& tm_kpool, const CUtensorMap& tm_vpool,

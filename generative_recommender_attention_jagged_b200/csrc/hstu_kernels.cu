@@ -20,74 +20,46 @@ namespace {
 constexpr long long kTsLimit = 1ll << 61;  // |timestamp| bound that keeps t_i + 1 - thr in range
 
 // ---------------------------------------------------------------------------
-// validate: one block per user
+// plan: validation by a grid of (user, part) blocks; the last block to finish
+// builds the work list, longest query blocks first
 // ---------------------------------------------------------------------------
-__global__ void validate_kernel(const AttnArgs a) {
-  const int u = blockIdx.x;
-  __shared__ int s_ok;
-  __shared__ int s_n, s_tso, s_pages;
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    const int q0 = a.q_offsets[u], q1 = a.q_offsets[u + 1];
-    if (u == 0 && q0 != 0) ok = 0;
-    if (u == a.B - 1 && q1 != a.T_q) ok = 0;
-    if (q0 < 0 || q1 < q0 || q1 > a.T_q) ok = 0;
-    const int L = a.paged ? a.cached_lens[u] : 0;
-    if (L < 0) ok = 0;
-    const long long n = (long long)L + (q1 - q0);
-    if (n > a.n_max) ok = 0;
-    const int c = a.num_cand ? a.num_cand[u] : 0;
-    if (c < 0 || c > q1 - q0) ok = 0;
-    int tso = q0, pages = 0;
-    if (a.paged) {
-      tso = a.ts_offsets[u];
-      if (u == 0 && tso != 0) ok = 0;
-      if ((long long)a.ts_offsets[u + 1] - tso != n) ok = 0;
-      pages = ceil_div(L, a.page_size);
-      if (pages > a.max_pages) ok = 0;
-    }
-    if (!ok) report_error(a.hdr, kErrLength, u);
-    s_ok = ok;
-    s_n = (int)n;
-    s_tso = tso;
-    s_pages = pages;
-  }
-  __syncthreads();
-  if (!s_ok) return;
-  if (a.paged) {
-    for (int x = threadIdx.x; x < s_pages; x += blockDim.x) {
-      const int pid = a.page_table[(size_t)u * a.max_pages + x];
-      if (pid < 0 || pid >= a.num_pages) report_error(a.hdr, kErrPage, u);
-    }
-  }
-  const int64_t* ts = a.ts + s_tso;
-  for (int j = threadIdx.x; j < s_n; j += blockDim.x) {
-    const long long t = ts[j];
-    if (t > kTsLimit || t < -kTsLimit || (j > 0 && t < ts[j - 1])) report_error(a.hdr, kErrUnsorted, u);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// schedule: one block builds the work list, longest query tiles first
-// ---------------------------------------------------------------------------
-constexpr int kSchedThreads = 1024;
+constexpr int kPlanThreads = 256;
 constexpr int kCostBins = 1024;
 
-__global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const AttnArgs a) {
-  __shared__ int hist[kCostBins];
-  __shared__ int start[kCostBins];
-  __shared__ int s_status;
+// checks of one user's offsets, lengths and candidate count (0 = bad)
+__device__ __forceinline__ int check_user(const AttnArgs& a, int u, int& n, int& tso, int& pages) {
+  int ok = 1;
+  const int q0 = a.q_offsets[u], q1 = a.q_offsets[u + 1];
+  if (u == 0 && q0 != 0) ok = 0;
+  if (u == a.B - 1 && q1 != a.T_q) ok = 0;
+  if (q0 < 0 || q1 < q0 || q1 > a.T_q) ok = 0;
+  const int L = a.paged ? a.cached_lens[u] : 0;
+  if (L < 0) ok = 0;
+  const long long nn = (long long)L + (q1 - q0);
+  if (nn > a.n_max) ok = 0;
+  const int c = a.num_cand ? a.num_cand[u] : 0;
+  if (c < 0 || c > q1 - q0) ok = 0;
+  tso = q0;
+  pages = 0;
+  if (a.paged) {
+    tso = a.ts_offsets[u];
+    if (u == 0 && tso != 0) ok = 0;
+    if ((long long)a.ts_offsets[u + 1] - tso != nn) ok = 0;
+    pages = ceil_div(L, a.page_size);
+    if (pages > a.max_pages) ok = 0;
+  }
+  n = (int)nn;
+  return ok;
+}
+
+// work list: per user, blocks of kItemRows query rows, each expanded to
+// H heads x num_splits splits; counting sort by cost (key tiles per split)
+__device__ void build_schedule(const AttnArgs& a, int* hist, int* start) {
   const int tid = threadIdx.x;
   for (int x = tid; x < kCostBins; x += blockDim.x) hist[x] = 0;
-  if (tid == 0) s_status = a.hdr->status;
   __syncthreads();
-  if (s_status != 0) {
-    if (tid == 0) a.hdr->n_items = 0;
-    return;
-  }
   const int per = a.H * a.num_splits;
   constexpr int tiles_per_item = kItemRows / kTile;
-  // cost of a block of query rows: key tiles of its longest tile, per split
   auto cost_of = [&](int user, int m) {
     const int nq = a.q_offsets[user + 1] - a.q_offsets[user];
     int c = 0;
@@ -129,6 +101,52 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const AttnArgs 
         }
     }
   }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const AttnArgs a, int parts, int schedule) {
+  const int u = blockIdx.x / parts;
+  const int part = blockIdx.x % parts;
+  __shared__ int s_ok, s_n, s_tso, s_pages, s_last;
+  __shared__ int hist[kCostBins];
+  __shared__ int start[kCostBins];
+  if (threadIdx.x == 0) {
+    int n, tso, pages;
+    const int ok = check_user(a, u, n, tso, pages);
+    if (!ok && part == 0) report_error(a.hdr, kErrLength, u);
+    s_ok = ok;
+    s_n = n;
+    s_tso = tso;
+    s_pages = pages;
+  }
+  __syncthreads();
+  if (s_ok) {
+    // this block's share of the user's page ids and timestamps
+    const int stride = blockDim.x * parts;
+    if (a.paged) {
+      for (int x = part * blockDim.x + threadIdx.x; x < s_pages; x += stride) {
+        const int pid = a.page_table[(size_t)u * a.max_pages + x];
+        if (pid < 0 || pid >= a.num_pages) report_error(a.hdr, kErrPage, u);
+      }
+    }
+    const int64_t* ts = a.ts + s_tso;
+    for (int j = part * blockDim.x + threadIdx.x; j < s_n; j += stride) {
+      const long long t = ts[j];
+      if (t > kTsLimit || t < -kTsLimit || (j > 0 && t < ts[j - 1])) report_error(a.hdr, kErrUnsorted, u);
+    }
+  }
+  if (!schedule) return;
+  // the last block to finish validating builds the work list (or an empty one)
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&a.hdr->blocks_done, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (*(volatile int32_t*)&a.hdr->status != 0) {
+    if (threadIdx.x == 0) a.hdr->n_items = 0;
+    return;
+  }
+  build_schedule(a, hist, start);
 }
 
 // ---------------------------------------------------------------------------
@@ -501,13 +519,10 @@ int num_sms() {
 
 }  // namespace
 
-cudaError_t launch_validate(const AttnArgs& a, cudaStream_t s) {
-  validate_kernel<<<a.B, 256, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_schedule(const AttnArgs& a, cudaStream_t s) {
-  schedule_kernel<<<1, kSchedThreads, 0, s>>>(a);
+cudaError_t launch_plan(const AttnArgs& a, bool schedule, int max_seq_len, cudaStream_t s) {
+  // enough blocks per user that a long user's timestamps are checked in parallel
+  const int parts = std::max(1, std::min(16, ceil_div(std::max(max_seq_len, 1), 1024)));
+  plan_kernel<<<a.B * parts, kPlanThreads, 0, s>>>(a, parts, schedule ? 1 : 0);
   return cudaGetLastError();
 }
 
