@@ -37,9 +37,12 @@ import synth  # noqa: E402
 FLOPS_PER_PAIR_HEAD = 2 * (128 + 128)  # QK^T and AV, d_qk = d_v = 128
 TILE = 128
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention-kernel launch
-# (per layer of this workload), from the ncu capture summarised in
-# profiles/attn_sm100_stack8.md; None until a capture of the current kernel exists.
-ATTN_TRAFFIC_BYTES = None
+# (one layer of this workload) and of one paged attention launch, from the ncu
+# captures summarised in profiles/attn_sm100_stack8.md and
+# profiles/attn_sm100_paged.md; set to None when the kernel changes until it
+# is captured again.
+ATTN_TRAFFIC_BYTES = 404_022_272 + 83_838_464
+PAGED_TRAFFIC_BYTES = 114_777_088 + 6_897_920
 
 
 def allowed_pairs(lengths, cands=None):
@@ -403,7 +406,7 @@ def run_paged_bench(args, device):
                          "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                          "frac": round(achieved / float(peaks["hbm_gbs"]), 4),
                          "peak_source": f"{kind} hbm_gbs", "bytes_per_launch": alg_bytes,
-                         "launch_ms": round(attn_ms, 4), "traffic": None}}
+                         "launch_ms": round(attn_ms, 4), "traffic": PAGED_TRAFFIC_BYTES}}
 
 
 # ----------------------------------------------------------------------------

@@ -58,6 +58,15 @@ __device__ __forceinline__ int bucket_of_dt(const long long* thr, long long dt) 
 // ---------------------------------------------------------------------------
 // geometry of a query tile (see TileGeom)
 // ---------------------------------------------------------------------------
+// key tiles needed by query tile `qtile` of a user with cached prefix L,
+// sequence length n and history h (pure arithmetic, no memory access)
+__host__ __device__ __forceinline__ int key_tiles_of(int L, int n, int h, int qtile) {
+  const int qs = L + qtile * kTile;
+  const int q_last = min(qs + kTile, n) - 1;
+  const int kv_end = max(0, min(q_last + 1, h));
+  return ceil_div(min(L, kv_end), kTile) + (kv_end > L ? ceil_div(kv_end - L, kTile) : 0);
+}
+
 __device__ __forceinline__ TileGeom tile_geom(const AttnArgs& a, int user, int qtile) {
   TileGeom g;
   const int q0 = a.q_offsets[user];

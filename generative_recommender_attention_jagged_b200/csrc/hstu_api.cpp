@@ -256,10 +256,11 @@ int32_t hstu_attn_paged_default_splits(const hstu_attn_params* p, int32_t max_ca
   if (check_params(p) != HSTU_OK) return 1;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long qtiles = (p->total_tokens + kItemRows - 1) / kItemRows;
-  const long long units = std::max<long long>(1, qtiles * p->num_heads);
+  // work items before splitting: every user has at least one block of query rows
+  const long long qblocks = std::max<long long>(p->batch, (p->total_tokens + kItemRows - 1) / kItemRows);
+  const long long units = std::max<long long>(1, qblocks * p->num_heads);
   const long long key_tiles = std::max(1, (max_cached_len + kTile - 1) / kTile);
-  long long s = (sms + units - 1) / units;          // at least one wave of CTAs
+  long long s = std::max<long long>(1, sms / units);  // fill one wave of CTAs, not more
   s = std::min<long long>(s, std::max<long long>(1, key_tiles / 2));  // >= 2 key tiles per split
   return (int32_t)std::max<long long>(1, std::min<long long>(s, kMaxSplits));
 }

@@ -60,16 +60,27 @@ __device__ void build_schedule(const AttnArgs& a, int* hist, int* start) {
   __syncthreads();
   const int per = a.H * a.num_splits;
   constexpr int tiles_per_item = kItemRows / kTile;
-  auto cost_of = [&](int user, int m) {
-    const int nq = a.q_offsets[user + 1] - a.q_offsets[user];
+  struct UserGeom {
+    int L, n, h, nq;
+  };
+  auto user_geom = [&](int u) {
+    UserGeom g;
+    g.nq = a.q_offsets[u + 1] - a.q_offsets[u];
+    g.L = a.paged ? a.cached_lens[u] : 0;
+    g.n = g.L + g.nq;
+    g.h = g.n - (a.num_cand ? a.num_cand[u] : 0);
+    return g;
+  };
+  // cost of a block of query rows: key tiles of its longest tile, per split
+  auto cost_of = [&](const UserGeom& g, int m) {
     int c = 0;
-    for (int x = 0; x < tiles_per_item && (m * tiles_per_item + x) * kTile < nq; ++x)
-      c = max(c, tile_geom(a, user, m * tiles_per_item + x).n_tiles);
+    for (int x = 0; x < tiles_per_item && (m * tiles_per_item + x) * kTile < g.nq; ++x)
+      c = max(c, key_tiles_of(g.L, g.n, g.h, m * tiles_per_item + x));
     return min(ceil_div(c, a.num_splits), kCostBins - 1);
   };
   for (int u = tid; u < a.B; u += blockDim.x) {
-    const int nq = a.q_offsets[u + 1] - a.q_offsets[u];
-    for (int m = ceil_div(nq, kItemRows) - 1; m >= 0; --m) atomicAdd(&hist[cost_of(u, m)], per);
+    const UserGeom g = user_geom(u);
+    for (int m = ceil_div(g.nq, kItemRows) - 1; m >= 0; --m) atomicAdd(&hist[cost_of(g, m)], per);
   }
   __syncthreads();
   // start[c] = number of items with a cost above c (descending order)
@@ -91,9 +102,9 @@ __device__ void build_schedule(const AttnArgs& a, int* hist, int* start) {
   }
   __syncthreads();
   for (int u = tid; u < a.B; u += blockDim.x) {
-    const int nq = a.q_offsets[u + 1] - a.q_offsets[u];
-    for (int m = ceil_div(nq, kItemRows) - 1; m >= 0; --m) {
-      const int pos = atomicAdd(&start[cost_of(u, m)], per);
+    const UserGeom g = user_geom(u);
+    for (int m = ceil_div(g.nq, kItemRows) - 1; m >= 0; --m) {
+      const int pos = atomicAdd(&start[cost_of(g, m)], per);
       for (int h = 0; h < a.H; ++h)
         for (int s = 0; s < a.num_splits; ++s) {
           const int idx = pos + h * a.num_splits + s;
