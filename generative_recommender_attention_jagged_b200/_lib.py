@@ -29,6 +29,8 @@ F_STAGE_PLAN = 0x10
 F_STAGE_ATTN = 0x20
 F_STAGE_EPILOGUE = 0x40
 
+LIN_SILU = 0x1
+
 
 class AttnParams(ctypes.Structure):
     _fields_ = [
@@ -43,6 +45,18 @@ class AttnParams(ctypes.Structure):
         ("u_stride", ctypes.c_int32),
         ("alpha", ctypes.c_float),
         ("ln_eps", ctypes.c_float),
+        ("dtype", ctypes.c_int32),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+class LinearParams(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_int64),
+        ("d_in", ctypes.c_int32),
+        ("d_out", ctypes.c_int32),
+        ("x_stride", ctypes.c_int64),
+        ("out_stride", ctypes.c_int64),
         ("dtype", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
     ]
@@ -83,6 +97,15 @@ def load() -> ctypes.CDLL:
     lib.hstu_check_device_error.restype = ctypes.c_int
     lib.hstu_status_string.argtypes = [ctypes.c_int]
     lib.hstu_status_string.restype = ctypes.c_char_p
+    LP = ctypes.POINTER(LinearParams)
+    lib.hstu_linear_workspace_size.argtypes = [LP]
+    lib.hstu_linear_workspace_size.restype = sz
+    for name in ("hstu_linear", "hstu_layer_f1", "hstu_layer_f2"):
+        fn = getattr(lib, name)
+        fn.argtypes = [LP, P, P, P, P, P, sz, P]
+        fn.restype = ctypes.c_int
+    lib.hstu_attn_fwd_static_ws.argtypes = [PP] + [P] * 13
+    lib.hstu_attn_fwd_static_ws.restype = ctypes.c_int
     lib.hstu_version.argtypes = []
     lib.hstu_version.restype = ctypes.c_int
     _lib = lib

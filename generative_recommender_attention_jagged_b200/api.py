@@ -199,12 +199,65 @@ def hstu_attn_fwd_static_ws(q, k, v, u, seq_offsets, timestamps, rab_pos, rab_ts
                          u_stride=us, ln_eps=ln_eps)
     if out is None:
         out = torch.empty(T, H * d, dtype=dt, device=q.device)
-    lib = _lib.load()
-    fn = lib.hstu_attn_fwd_static_ws
-    fn.argtypes = [ctypes.POINTER(_lib.AttnParams)] + [ctypes.c_void_p] * 13
-    fn.restype = ctypes.c_int
-    rc = fn(ctypes.byref(params), _p(q), _p(k), _p(v), _p(u), _p(seq_offsets), _p(timestamps),
+    rc = _lib.load().hstu_attn_fwd_static_ws(ctypes.byref(params), _p(q), _p(k), _p(v), _p(u), _p(seq_offsets), _p(timestamps),
             _p(num_candidates), _p(rab_pos), _p(rab_ts), _p(ln_gamma), _p(ln_beta), _p(out),
             _stream(stream))
     _lib.check(rc, "hstu_attn_fwd_static_ws")
     return out
+
+
+def linear_params(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor, silu: bool) -> _lib.LinearParams:
+    return _lib.LinearParams(rows=x.shape[0], d_in=x.shape[1], d_out=w.shape[1],
+                             x_stride=x.stride(0) if x.shape[0] > 1 else x.shape[1],
+                             out_stride=out.stride(0) if out.shape[0] > 1 else out.shape[1],
+                             dtype=_DT[x.dtype], flags=_lib.LIN_SILU if silu else 0)
+
+
+def hstu_linear_workspace_size(p: Optional[_lib.LinearParams] = None) -> int:
+    p = p if p is not None else _lib.LinearParams()
+    return int(_lib.load().hstu_linear_workspace_size(ctypes.byref(p)))
+
+
+def _linear(name: str, x, w, bias, out, workspace, stream, silu: bool):
+    for nm, t in (("x", x), ("w", w), ("out", out)):
+        _need_cuda(nm, t, x.dtype)
+    _need_cuda("bias", bias, torch.float32)
+    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[0]:
+        raise ValueError(f"{name}: x [T, d_in] and w [d_in, d_out] expected")
+    if x.stride(1) != 1 or not w.is_contiguous():
+        raise ValueError(f"{name}: x rows and w must be contiguous")
+    if out is None:
+        out = torch.empty(x.shape[0], w.shape[1], dtype=x.dtype, device=x.device)
+    if out.dim() != 2 or out.shape != (x.shape[0], w.shape[1]) or out.stride(1) != 1:
+        raise ValueError(f"{name}: out [T, d_out] with contiguous rows expected")
+    p = linear_params(x, w, out, silu)
+    if workspace is None:
+        workspace = torch.empty(hstu_linear_workspace_size(p), dtype=torch.uint8, device=x.device)
+    rc = getattr(_lib.load(), name)(ctypes.byref(p), _p(x), _p(w), _p(bias), _p(out), _p(workspace),
+                                    workspace.numel(), _stream(stream))
+    _lib.check(rc, name)
+    return out
+
+
+def hstu_layer_f1(x, w1, b1=None, *, out=None, workspace=None, stream=None):
+    """[U | V | Q | K] = SiLU(x W1 + b1) as one [T, 4*H*d] tensor (blocks head-major)."""
+    return _linear("hstu_layer_f1", x, w1, b1, out, workspace, stream, True)
+
+
+def hstu_layer_f2(y, w2, b2=None, *, out=None, workspace=None, stream=None):
+    """x_next = y W2 + b2."""
+    return _linear("hstu_layer_f2", y, w2, b2, out, workspace, stream, False)
+
+
+def hstu_linear(x, w, bias=None, *, silu: bool = False, out=None, workspace=None, stream=None):
+    """out = act(x W + bias), act = SiLU or identity."""
+    return _linear("hstu_linear", x, w, bias, out, workspace, stream, silu)
+
+
+def split_uvqk(uvqk: torch.Tensor, num_heads: int, head_dim: int):
+    """Views u [T, H*d] and v, q, k [T, H, d] of f1's [T, 4*H*d] output (no copy)."""
+    hd = num_heads * head_dim
+    T = uvqk.shape[0]
+    u = uvqk[:, 0:hd]
+    v, q, k = (uvqk[:, b * hd:(b + 1) * hd].unflatten(1, (num_heads, head_dim)) for b in (1, 2, 3))
+    return u, v, q, k

@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhstu.so")
-SOURCES = ["hstu_api.cpp", "ts_table.cpp", "hstu_kernels.cu", "attn_sm100.cu", "hstu_static_ws.cu"]
+SOURCES = ["hstu_api.cpp", "ts_table.cpp", "hstu_kernels.cu", "attn_sm100.cu", "hstu_static_ws.cu", "hstu_linear.cu"]
 HEADERS = ["hstu_internal.h", "device_common.cuh"]
 
 
@@ -36,7 +36,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "-shared",
            "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           "-o", tmp] + [os.path.join(CSRC, f) for f in SOURCES] + ["-lquadmath"]
+           "-o", tmp] + [os.path.join(CSRC, f) for f in SOURCES] + ["-lquadmath", "-lcublasLt"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)

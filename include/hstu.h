@@ -34,7 +34,8 @@
  *
  * Conventions
  *   - The caller owns every buffer.  The library never allocates device or
- *     host memory; scratch space is the caller's `workspace`.
+ *     host memory; scratch space is the caller's `workspace` (the one
+ *     exception, cuBLASLt's per-device handle, is described at hstu_linear).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  The return value covers host-side argument checks and
  *     launch errors only.  Errors the device detects (bad offsets, lengths
@@ -197,6 +198,59 @@ int hstu_attn_fwd_paged(const hstu_attn_params* p, const void* q_new, const void
  */
 int hstu_ts_bucket(const int64_t* dt, int64_t n, int32_t num_buckets, int32_t* out,
                    hstu_stream_t stream);
+
+/* ---- Layer glue around the attention ------------------------------------
+ *
+ * One HSTU layer is  x -> f1 -> attention -> f2  (no residual, no input norm):
+ *   f1:  [U | V | Q | K] = SiLU(x W1 + b1)       d_model -> 4*H*d
+ *   f2:  x_next          = y W2 + b2             H*d -> d_model
+ * ("Generative Recommenders at Scale", Inside NVIDIA's GPU-native stack: the
+ * pointwise projection with SiLU feeding the attention; "How Generative
+ * Recommenders Are Redefining RecSys at Scale", Takeaways: gating before the
+ * output projection.)  f1's output columns are ordered [U | V | Q | K], each
+ * block H*d wide and head-major inside (column = block*H*d + head*d + e), so
+ * the four blocks of one [T, 4*H*d] buffer are directly the u, v, q, k
+ * arguments of hstu_attn_fwd (token stride 4*H*d).
+ *
+ * Both are plain GEMMs (cuBLASLt, fp32 accumulate, bias added in the GEMM
+ * epilogue); f1's SiLU runs in place right after it in one vectorised kernel.
+ * The first call on a device creates that device's cuBLASLt handle (host
+ * memory owned by cuBLASLt); nothing else is allocated.
+ */
+#define HSTU_LIN_SILU 0x1u  /* hstu_linear only: apply SiLU to the output (f1) */
+
+typedef struct {
+  int64_t rows;        /* T (0 is allowed: nothing to do)                              */
+  int32_t d_in;        /* K: columns of x, rows of w                                   */
+  int32_t d_out;       /* N: columns of w and of out; a multiple of 8                   */
+  int64_t x_stride;    /* elements between rows of x; 0 = d_in; a multiple of 8        */
+  int64_t out_stride;  /* elements between rows of out; 0 = d_out; a multiple of 8     */
+  hstu_dtype dtype;    /* x, w, out: bf16 (fp32 accumulate) or fp32                     */
+  uint32_t flags;      /* HSTU_LIN_SILU or 0                                            */
+} hstu_linear_params;
+
+/* Bytes of workspace the linear entry points use: cuBLASLt scratch (32 MiB)
+ * plus room for the bf16 copy of the bias. */
+size_t hstu_linear_workspace_size(const hstu_linear_params* p);
+
+/* out[r, :] = act(x[r, :] W + bias), act = SiLU with HSTU_LIN_SILU, else identity.
+ *   x    [rows, d_in]  dtype, row stride x_stride, device, 16-byte aligned
+ *   w    [d_in, d_out] dtype, row-major, contiguous, device, 16-byte aligned
+ *   bias [d_out] fp32 device or NULL (= 0); for bf16 it is rounded to bf16 into
+ *        the workspace and added to the fp32 accumulator in the GEMM epilogue
+ *   out  [rows, d_out] dtype, row stride out_stride; must not overlap x or w
+ * Returns HSTU_OK, HSTU_ERR_INVALID_ARG / _ALIGNMENT / _WORKSPACE for bad
+ * arguments (nothing launched), HSTU_ERR_CUDA if cuBLASLt or a launch fails. */
+int hstu_linear(const hstu_linear_params* p, const void* x, const void* w, const float* bias, void* out,
+                void* workspace, size_t workspace_bytes, hstu_stream_t stream);
+
+/* f1 of the layer: hstu_linear with HSTU_LIN_SILU forced on (w = W1 [d_model, 4*H*d]). */
+int hstu_layer_f1(const hstu_linear_params* p, const void* x, const void* w1, const float* b1, void* uvqk,
+                  void* workspace, size_t workspace_bytes, hstu_stream_t stream);
+
+/* f2 of the layer: hstu_linear without activation (w = W2 [H*d, d_model]). */
+int hstu_layer_f2(const hstu_linear_params* p, const void* y, const void* w2, const float* b2, void* x_next,
+                  void* workspace, size_t workspace_bytes, hstu_stream_t stream);
 
 /* Synchronises `stream`, then returns the status word the device wrote into
  * `workspace` during the last call that used it (HSTU_OK if none). */

@@ -115,3 +115,38 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         hstu.hstu_attn_fwd(q, q, q, q.view(4, 128), torch.tensor([0, 4], dtype=torch.int32),
                            torch.zeros(4, dtype=torch.int64), torch.zeros(7), torch.zeros(128), n_max=4)
+
+
+# ---- linear glue (f1 / f2) --------------------------------------------------
+def test_linear_params_struct_matches_header(lib):
+    # int64 rows, int32 d_in, int32 d_out, int64 x_stride, int64 out_stride, int32 dtype, uint32 flags
+    assert ctypes.sizeof(_lib.LinearParams) == 40
+
+
+def lin(**kw):
+    base = dict(rows=300, d_in=512, d_out=2048, x_stride=0, out_stride=0, dtype=_lib.DT_BF16, flags=0)
+    base.update(kw)
+    return _lib.LinearParams(**base)
+
+
+@pytest.mark.parametrize("name", ["hstu_linear", "hstu_layer_f1", "hstu_layer_f2"])
+def test_linear_rejects_bad_args_on_host(lib, name):
+    fn = getattr(lib, name)
+    a = ctypes.c_void_p(0x1000)
+    ws = 1 << 26
+    assert fn(None, a, a, None, a, a, ws, None) == -1
+    assert fn(ctypes.byref(lin(rows=-1)), a, a, None, a, a, ws, None) == -1
+    assert fn(ctypes.byref(lin(d_in=0)), a, a, None, a, a, ws, None) == -1
+    assert fn(ctypes.byref(lin(dtype=7)), a, a, None, a, a, ws, None) == -1
+    assert fn(ctypes.byref(lin(flags=0x8)), a, a, None, a, a, ws, None) == -1
+    assert fn(ctypes.byref(lin(x_stride=100)), a, a, None, a, a, ws, None) == -1   # stride < d_in
+    assert fn(ctypes.byref(lin()), None, a, None, a, a, ws, None) == -1
+    assert fn(ctypes.byref(lin(d_out=2044)), a, a, None, a, a, ws, None) == -3
+    assert fn(ctypes.byref(lin()), ctypes.c_void_p(0x1008), a, None, a, a, ws, None) == -3
+    assert fn(ctypes.byref(lin()), a, a, None, a, a, 1024, None) == -5
+    # no rows: nothing to do, no pointer is looked at
+    assert fn(ctypes.byref(lin(rows=0)), None, None, None, None, None, 0, None) == 0
+
+
+def test_linear_workspace_size(lib):
+    assert hstu.hstu_linear_workspace_size() >= 1 << 20
