@@ -320,7 +320,8 @@ def run_ours(args, rank, world, device):
         "dtype": "bf16",
         "data": "synthetic (seeded; no dataset)",
         "config": {"workload": f"{args.workload}: 8-layer HSTU attention, B={b0.batch} users, lengths "
-                               f"U[4160,8320] (T={T}), H={H}, d={d}, N_max={b0.n_max}, causal",
+                               f"{'all 8192' if args.workload == 'stack8_n8192' else 'U[4160,8320]'} "
+                               f"(T={T}), H={H}, d={d}, N_max={b0.n_max}, causal",
                    "global_batch": b0.batch * world, "total_tokens_per_gpu": T, "layers": L,
                    "parallelism": f"replicas x{world} (users sharded, no collective)",
                    "l2": "inputs larger than L2 (8 per-layer Q/K/V/U sets, %.2f GB)" %
@@ -329,7 +330,8 @@ def run_ours(args, rank, world, device):
         "roofline": {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)",
-                     "traffic": ATTN_TRAFFIC_BYTES,
+                     # measured on the default workload's layer-0 launch; none for other workloads
+                     "traffic": ATTN_TRAFFIC_BYTES if args.workload == "stack8_bf16" else None,
                      "launch_ms": round(attn_avg_ms, 4), "flops_per_launch": flops_layer,
                      "issued_tile_tflops": round(issued_tflops, 2),
                      "issued_frac": round(issued_tflops / peak, 4)},
@@ -409,6 +411,54 @@ def run_paged_bench(args, device):
                          "launch_ms": round(attn_ms, 4), "traffic": PAGED_TRAFFIC_BYTES}}
 
 
+def run_glue_bench(args, device):
+    """The layer glue around the attention at the 8-layer stack's shapes:
+    f1 = SiLU(x W1 + b1) (512 -> 2048, cuBLASLt GEMM + in-place SiLU kernel)
+    and f2 = y W2 + b2 (512 -> 512).  Two input sets alternate so that the
+    operands (~270 MB per f1 call) do not sit in L2 between calls."""
+    import generative_recommender_attention_jagged_b200 as hstu
+    s = synth.workload_stack("stack8_bf16", num_layers=1)
+    T = s.x.shape[0]
+    _, _, w = s.layers[0]
+    w1 = to_dev(torch.from_numpy(w.w1).to(torch.bfloat16))
+    w2 = to_dev(torch.from_numpy(w.w2).to(torch.bfloat16))
+    b1, b2 = to_dev(w.b1, torch.float32), to_dev(w.b2, torch.float32)
+    xs = [to_dev(s.x), to_dev(s.x).roll(1, 0).contiguous()]
+    zs = [torch.empty(T, 2048, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    ys = [z[:, :512] for z in zs]          # a [T, 512] view with row stride 2048, as f2 sees y after attention
+    outs = [torch.empty(T, 512, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    ws = torch.empty(hstu.hstu_linear_workspace_size(hstu.api.linear_params(xs[0], w1, zs[0], True)),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    steps = max(3, min(args.steps, 50))
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(steps):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    f1_ms = timed(lambda i: hstu.hstu_layer_f1(xs[i % 2], w1, b1, out=zs[i % 2], workspace=ws))
+    f2_ms = timed(lambda i: hstu.hstu_layer_f2(ys[i % 2], w2, b2, out=outs[i % 2], workspace=ws))
+    peaks, kind = measured_peaks()
+    f1_flops, f2_flops = 2.0 * T * 512 * 2048, 2.0 * T * 512 * 512
+    f1_tf, f2_tf = f1_flops / (f1_ms * 1e-3) / 1e12, f2_flops / (f2_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    return {"workload": f"stack8_bf16 layer glue: T={T}, f1 512->2048 + SiLU, f2 512->512, bf16",
+            "f1_ms": round(f1_ms, 4), "f2_ms": round(f2_ms, 4),
+            "f1_tflops": round(f1_tf, 1), "f2_tflops": round(f2_tf, 1),
+            "roofline": {"kernel": "cuBLASLt GEMM (+ SiLU pass for f1)", "bound": "tensor",
+                         "achieved": round(f1_tf, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(f1_tf / peak, 4), "peak_source": f"{kind} bf16_tflops (burst)",
+                         "traffic": None}}
+
+
 # ----------------------------------------------------------------------------
 # reference arm: the fp64 CPU oracle on the host cores
 # ----------------------------------------------------------------------------
@@ -451,6 +501,7 @@ def main():
     ap.add_argument("--workload", default="stack8_bf16", choices=["stack8_bf16", "stack8_n8192"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-paged", action="store_true")
+    ap.add_argument("--no-glue", action="store_true", help="skip the f1/f2 layer-glue timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--paged-only", action="store_true",
                     help="run only the paged incremental sub-benchmark (profiling captures)")
@@ -483,6 +534,8 @@ def main():
     result, b0 = run_ours(args, rank, world, device)
     if rank == 0 and not args.no_paged and world == 1:
         result["paged"] = run_paged_bench(args, device)
+    if rank == 0 and not args.no_glue and world == 1:
+        result["glue"] = run_glue_bench(args, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
