@@ -16,7 +16,7 @@ HSTU_OK = 0
 STATUS_NAMES = {
     0: "HSTU_OK", -1: "HSTU_ERR_INVALID_ARG", -2: "HSTU_ERR_UNSUPPORTED", -3: "HSTU_ERR_ALIGNMENT",
     -4: "HSTU_ERR_LENGTH", -5: "HSTU_ERR_WORKSPACE", -6: "HSTU_ERR_CUDA", -7: "HSTU_ERR_TIMEOUT",
-    -8: "HSTU_ERR_UNSORTED", -9: "HSTU_ERR_PAGE",
+    -8: "HSTU_ERR_UNSORTED", -9: "HSTU_ERR_PAGE", -10: "HSTU_ERR_POOL",
 }
 
 DT_F32 = 0
@@ -59,6 +59,20 @@ class LinearParams(ctypes.Structure):
         ("out_stride", ctypes.c_int64),
         ("dtype", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
+    ]
+
+
+class KvParams(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("max_pages_per_user", ctypes.c_int32),
+        ("kv_stride", ctypes.c_int32),
+        ("total_new", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
     ]
 
 
@@ -106,6 +120,13 @@ def load() -> ctypes.CDLL:
         fn.restype = ctypes.c_int
     lib.hstu_attn_fwd_static_ws.argtypes = [PP] + [P] * 13
     lib.hstu_attn_fwd_static_ws.restype = ctypes.c_int
+    KP = ctypes.POINTER(KvParams)
+    lib.hstu_kv_workspace_size.argtypes = [KP]
+    lib.hstu_kv_workspace_size.restype = sz
+    lib.hstu_kv_append.argtypes = [KP] + [P] * 11 + [sz, P]
+    lib.hstu_kv_append.restype = ctypes.c_int
+    lib.hstu_kv_evict.argtypes = [KP] + [P] * 6 + [sz, P]
+    lib.hstu_kv_evict.restype = ctypes.c_int
     lib.hstu_version.argtypes = []
     lib.hstu_version.restype = ctypes.c_int
     _lib = lib

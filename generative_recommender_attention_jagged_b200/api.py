@@ -261,3 +261,62 @@ def split_uvqk(uvqk: torch.Tensor, num_heads: int, head_dim: int):
     u = uvqk[:, 0:hd]
     v, q, k = (uvqk[:, b * hd:(b + 1) * hd].unflatten(1, (num_heads, head_dim)) for b in (1, 2, 3))
     return u, v, q, k
+
+
+def kv_params(k_pool: torch.Tensor, page_table: torch.Tensor, k_new: Optional[torch.Tensor] = None) -> _lib.KvParams:
+    num_pages, H, P, d = k_pool.shape
+    stride = 0 if k_new is None or k_new.shape[0] <= 1 else k_new.stride(0)
+    return _lib.KvParams(batch=page_table.shape[0], num_heads=H, head_dim=d, page_size=P, num_pages=num_pages,
+                         max_pages_per_user=page_table.shape[1], kv_stride=stride,
+                         total_new=0 if k_new is None else k_new.shape[0], dtype=_DT[k_pool.dtype])
+
+
+def hstu_kv_workspace_size(p: _lib.KvParams) -> int:
+    return int(_lib.load().hstu_kv_workspace_size(ctypes.byref(p)))
+
+
+def _kv_check(k_pool, page_table, cached_lens, free_pages, free_count):
+    _need_cuda("k_pool", k_pool)
+    for name, t in (("page_table", page_table), ("cached_lens", cached_lens), ("free_pages", free_pages),
+                    ("free_count", free_count)):
+        _need_cuda(name, t, torch.int32)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not k_pool.is_contiguous():
+        raise ValueError("k_pool must be contiguous")
+
+
+def hstu_kv_append(k_new, v_new, new_offsets, k_pool, v_pool, page_table, cached_lens, free_pages, free_count, *,
+                   num_append=None, workspace=None, stream=None):
+    """Appends the first num_append[u] new tokens of every user (all when None)
+    behind its cached prefix, taking pages from the free stack; in place."""
+    _kv_check(k_pool, page_table, cached_lens, free_pages, free_count)
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("v_pool", v_pool)):
+        _need_cuda(name, t, k_pool.dtype)
+    _need_cuda("new_offsets", new_offsets, torch.int32)
+    _need_cuda("num_append", num_append, torch.int32)
+    if k_new.stride() != v_new.stride() or k_new.stride(2) != 1 or k_new.stride(1) != k_new.shape[2]:
+        raise ValueError("k_new and v_new must be [T, H, d] views with packed heads and one token stride")
+    p = kv_params(k_pool, page_table, k_new)
+    if workspace is None:
+        workspace = torch.empty(hstu_kv_workspace_size(p), dtype=torch.uint8, device=k_pool.device)
+    rc = _lib.load().hstu_kv_append(ctypes.byref(p), _p(k_new), _p(v_new), _p(new_offsets), _p(num_append),
+                                    _p(k_pool), _p(v_pool), _p(page_table), _p(cached_lens), _p(free_pages),
+                                    _p(free_count), _p(workspace), workspace.numel(), _stream(stream))
+    _lib.check(rc, "hstu_kv_append")
+    return workspace
+
+
+def hstu_kv_evict(evict_mask, k_pool, page_table, cached_lens, free_pages, free_count, *, workspace=None,
+                  stream=None):
+    """Returns the pages of every user with evict_mask[u] != 0 to the free stack; in place."""
+    _kv_check(k_pool, page_table, cached_lens, free_pages, free_count)
+    _need_cuda("evict_mask", evict_mask, torch.int32)
+    p = kv_params(k_pool, page_table)
+    if workspace is None:
+        workspace = torch.empty(hstu_kv_workspace_size(p), dtype=torch.uint8, device=k_pool.device)
+    rc = _lib.load().hstu_kv_evict(ctypes.byref(p), _p(evict_mask), _p(page_table), _p(cached_lens),
+                                   _p(free_pages), _p(free_count), _p(workspace), workspace.numel(),
+                                   _stream(stream))
+    _lib.check(rc, "hstu_kv_evict")
+    return workspace

@@ -356,6 +356,7 @@ const char* hstu_status_string(int status) {
     case HSTU_ERR_TIMEOUT: return "HSTU_ERR_TIMEOUT: a device wait ran out";
     case HSTU_ERR_UNSORTED: return "HSTU_ERR_UNSORTED: timestamps decrease within a user or exceed 2^61";
     case HSTU_ERR_PAGE: return "HSTU_ERR_PAGE: page id out of range";
+    case HSTU_ERR_POOL: return "HSTU_ERR_POOL: free-page stack or page-table row too small";
     default: return "unknown status";
   }
 }

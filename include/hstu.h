@@ -76,7 +76,9 @@ typedef enum {
   HSTU_ERR_CUDA = -6,          /* a CUDA runtime/driver call failed                          */
   HSTU_ERR_TIMEOUT = -7,       /* device: a bounded wait inside a kernel ran out             */
   HSTU_ERR_UNSORTED = -8,      /* device: timestamps decrease inside a user                  */
-  HSTU_ERR_PAGE = -9           /* device: a page-table entry outside [0, num_pages)          */
+  HSTU_ERR_PAGE = -9,          /* device: a page-table entry outside [0, num_pages)          */
+  HSTU_ERR_POOL = -10          /* device: KV append found the free-page stack or a page-table
+                                  row too small; nothing was changed                         */
 } hstu_status;
 
 typedef enum { HSTU_DT_F32 = 0, HSTU_DT_BF16 = 1 } hstu_dtype;
@@ -251,6 +253,61 @@ int hstu_layer_f1(const hstu_linear_params* p, const void* x, const void* w1, co
 /* f2 of the layer: hstu_linear without activation (w = W2 [H*d, d_model]). */
 int hstu_layer_f2(const hstu_linear_params* p, const void* y, const void* w2, const float* b2, void* x_next,
                   void* workspace, size_t workspace_bytes, hstu_stream_t stream);
+
+/* ---- Paged KV cache: the write side --------------------------------------
+ *
+ * ("Recomendador generativo HSTU com Dynamo-Triton", KV cache section: the
+ * attention state of a user's stable prefix is kept in a paged GPU table, so
+ * that a request only computes its new actions and candidates.)  These calls
+ * maintain that table after a request: the new actions' K and V are appended
+ * behind the cached prefix (candidates are never cached), pages come from a
+ * free-page stack on the device, and evicting a user returns its pages.
+ *
+ * Pool and table have the layout hstu_attn_fwd_paged reads:
+ *   k_pool, v_pool  [num_pages, H, page_size, d] dtype
+ *   page_table      [batch, max_pages_per_user] int32; entries past a user's
+ *                   last page are -1 (append writes new ids, evict writes -1)
+ *   cached_lens     [batch] int32 tokens cached per user
+ *   free_pages      [num_pages] int32 stack of free page ids; the top
+ *                   free_count[0] entries (indices 0 .. free_count-1) are free
+ *   free_count      [1] int32 device
+ * Allocation policy (deterministic): users take pages in user order from the
+ * top of the stack; user u's j-th new page is
+ *   free_pages[free_count - 1 - (pages taken by users < u) - j].
+ * Both calls are all-or-nothing: if the stack or a page-table row is too
+ * small for the whole batch, the device writes HSTU_ERR_POOL to the status
+ * word of `workspace` (hstu_check_device_error) and changes nothing.
+ */
+typedef struct {
+  int32_t batch;               /* users in page_table / cached_lens                        */
+  int32_t num_heads, head_dim; /* H, d of the pool                                         */
+  int32_t page_size;           /* tokens per page (any positive value)                     */
+  int32_t num_pages;           /* pages in the pool                                        */
+  int32_t max_pages_per_user;  /* columns of page_table                                    */
+  int32_t kv_stride;           /* elements between tokens of k_new / v_new; 0 = H*d         */
+  int32_t total_new;           /* rows of k_new / v_new (new_offsets[batch] must not exceed) */
+  hstu_dtype dtype;            /* element type of the pool and of k_new / v_new            */
+} hstu_kv_params;
+
+/* Bytes of workspace hstu_kv_append / hstu_kv_evict need (status word + per-user scratch). */
+size_t hstu_kv_workspace_size(const hstu_kv_params* p);
+
+/* Append: for user u the first num_append[u] of its new tokens (rows
+ * new_offsets[u] .. of k_new / v_new [T_new, H, d]) go to positions
+ * cached_lens[u] .. of its sequence; then cached_lens[u] += num_append[u].
+ * num_append NULL = all new tokens.  Pointers are device pointers; k_new,
+ * v_new, the pools and kv_stride * element size must be 16-byte aligned. */
+int hstu_kv_append(const hstu_kv_params* p, const void* k_new, const void* v_new, const int32_t* new_offsets,
+                   const int32_t* num_append, void* k_pool, void* v_pool, int32_t* page_table,
+                   int32_t* cached_lens, int32_t* free_pages, int32_t* free_count, void* workspace,
+                   size_t workspace_bytes, hstu_stream_t stream);
+
+/* Evict: every user u with evict_mask[u] != 0 pushes its pages back onto the
+ * free stack (in page-table order), gets a row of -1 and cached_lens[u] = 0.
+ * The pool contents are left as they are. */
+int hstu_kv_evict(const hstu_kv_params* p, const int32_t* evict_mask, int32_t* page_table, int32_t* cached_lens,
+                  int32_t* free_pages, int32_t* free_count, void* workspace, size_t workspace_bytes,
+                  hstu_stream_t stream);
 
 /* Synchronises `stream`, then returns the status word the device wrote into
  * `workspace` during the last call that used it (HSTU_OK if none). */

@@ -51,7 +51,7 @@ def test_params_struct_matches_header(lib):
 
 def test_status_strings(lib):
     assert hstu.hstu_status_string(0) == "HSTU_OK"
-    for code in range(-9, 0):
+    for code in range(-10, 0):
         assert hstu.hstu_status_string(code).startswith(_lib.STATUS_NAMES[code])
     assert hstu.hstu_version() == 100
 
@@ -150,3 +150,32 @@ def test_linear_rejects_bad_args_on_host(lib, name):
 
 def test_linear_workspace_size(lib):
     assert hstu.hstu_linear_workspace_size() >= 1 << 20
+
+
+# ---- KV cache write side ----------------------------------------------------
+def test_kv_params_struct_matches_header(lib):
+    assert ctypes.sizeof(_lib.KvParams) == 9 * 4
+
+
+def kvp(**kw):
+    base = dict(batch=3, num_heads=4, head_dim=128, page_size=32, num_pages=100, max_pages_per_user=8,
+                kv_stride=0, total_new=50, dtype=_lib.DT_BF16)
+    base.update(kw)
+    return _lib.KvParams(**base)
+
+
+def test_kv_rejects_bad_args_on_host(lib):
+    a = ctypes.c_void_p(0x1000)
+    ws = 1 << 20
+    assert lib.hstu_kv_workspace_size(ctypes.byref(kvp())) >= 256 + 3 * 8
+    assert lib.hstu_kv_workspace_size(ctypes.byref(kvp(batch=0))) == 0
+    assert lib.hstu_kv_append(None, *([a] * 11), ws, None) == -1
+    assert lib.hstu_kv_append(ctypes.byref(kvp(page_size=0)), *([a] * 11), ws, None) == -1
+    assert lib.hstu_kv_append(ctypes.byref(kvp(dtype=5)), *([a] * 11), ws, None) == -1
+    assert lib.hstu_kv_append(ctypes.byref(kvp()), None, *([a] * 10), ws, None) == -1
+    assert lib.hstu_kv_append(ctypes.byref(kvp(kv_stride=100)), *([a] * 11), ws, None) == -1  # < H*d
+    assert lib.hstu_kv_append(ctypes.byref(kvp(head_dim=4)), *([a] * 11), ws, None) == -3      # 8-byte rows
+    assert lib.hstu_kv_append(ctypes.byref(kvp()), ctypes.c_void_p(0x1004), *([a] * 10), ws, None) == -3
+    assert lib.hstu_kv_append(ctypes.byref(kvp()), *([a] * 11), 16, None) == -5
+    assert lib.hstu_kv_evict(ctypes.byref(kvp()), None, a, a, a, a, a, ws, None) == -1
+    assert lib.hstu_kv_evict(ctypes.byref(kvp()), *([a] * 6), 16, None) == -5
