@@ -23,6 +23,8 @@ from .api import (  # noqa: F401
     hstu_layer_f2,
     hstu_linear,
     hstu_linear_workspace_size,
+    hstu_mfalcon_fwd,
+    hstu_mfalcon_workspace_size,
     hstu_ts_bucket,
     hstu_version,
     split_uvqk,
@@ -33,5 +35,6 @@ __all__ = [
     "hstu_attn_paged_default_splits", "hstu_attn_paged_workspace_size", "hstu_attn_workspace_size",
     "hstu_check_device_error", "hstu_status_string", "hstu_ts_bucket", "hstu_version",
     "hstu_layer_f1", "hstu_layer_f2", "hstu_linear", "hstu_linear_workspace_size", "split_uvqk",
-    "hstu_kv_append", "hstu_kv_evict", "hstu_kv_workspace_size",
+    "hstu_kv_append", "hstu_kv_evict", "hstu_kv_workspace_size", "hstu_mfalcon_fwd",
+    "hstu_mfalcon_workspace_size",
 ]

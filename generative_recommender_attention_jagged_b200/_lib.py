@@ -120,6 +120,11 @@ def load() -> ctypes.CDLL:
         fn.restype = ctypes.c_int
     lib.hstu_attn_fwd_static_ws.argtypes = [PP] + [P] * 13
     lib.hstu_attn_fwd_static_ws.restype = ctypes.c_int
+    lib.hstu_mfalcon_workspace_size.argtypes = [PP, i32, i32, i64]
+    lib.hstu_mfalcon_workspace_size.restype = sz
+    lib.hstu_mfalcon_fwd.argtypes = ([PP] + [P] * 7 + [i64, P] + [P] * 6 + [i32, P, i32, i32, P, i32, i32, i32, P, P,
+                                                                         sz, P])
+    lib.hstu_mfalcon_fwd.restype = ctypes.c_int
     KP = ctypes.POINTER(KvParams)
     lib.hstu_kv_workspace_size.argtypes = [KP]
     lib.hstu_kv_workspace_size.restype = sz

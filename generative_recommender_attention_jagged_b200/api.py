@@ -320,3 +320,54 @@ def hstu_kv_evict(evict_mask, k_pool, page_table, cached_lens, free_pages, free_
                                    _stream(stream))
     _lib.check(rc, "hstu_kv_evict")
     return workspace
+
+
+def hstu_mfalcon_workspace_size(p: _lib.AttnParams, microbatch: int, num_splits: int, hist_tokens: int) -> int:
+    return int(_lib.load().hstu_mfalcon_workspace_size(ctypes.byref(p), microbatch, num_splits, hist_tokens))
+
+
+def hstu_mfalcon_fwd(q_c, k_c, v_c, u_c, cand_offsets, hist_timestamps, hist_ts_offsets, cand_timestamps,
+                     rab_pos, rab_ts, k_pool, v_pool, kv_page_table, cached_lens, *, n_max: int, microbatch: int,
+                     max_candidates: int, max_cached_len: Optional[int] = None, alpha: Optional[float] = None,
+                     ln_gamma=None, ln_beta=None, ln_eps: float = 1e-5, num_splits: Optional[int] = None,
+                     out=None, workspace=None, force_simt: bool = False, precise_silu: bool = False,
+                     stream=None):
+    """M-FALCON: every candidate attends to its user's cached history and itself;
+    candidates go through the paged forward `microbatch` per user at a time."""
+    T, H, d = q_c.shape
+    dt = q_c.dtype
+    for name, t in (("q_c", q_c), ("k_c", k_c), ("v_c", v_c), ("u_c", u_c), ("k_pool", k_pool), ("v_pool", v_pool)):
+        _need_cuda(name, t, dt)
+    for name, t in (("cand_offsets", cand_offsets), ("hist_ts_offsets", hist_ts_offsets),
+                    ("kv_page_table", kv_page_table), ("cached_lens", cached_lens)):
+        _need_cuda(name, t, torch.int32)
+    _need_cuda("hist_timestamps", hist_timestamps, torch.int64)
+    _need_cuda("cand_timestamps", cand_timestamps, torch.int64)
+    qs = _rows_view("q_c", q_c, H, d)
+    if _rows_view("k_c", k_c, H, d) != qs or _rows_view("v_c", v_c, H, d) != qs:
+        raise ValueError("q_c, k_c and v_c must share one token stride")
+    us = _rows_view("u_c", u_c, H, d)
+    B = cand_offsets.numel() - 1
+    num_pages, _, page_size, _ = k_pool.shape
+    mc = n_max if max_cached_len is None else max_cached_len
+    flags = (_lib.F_FORCE_SIMT if force_simt else 0) | (_lib.F_PRECISE_SILU if precise_silu else 0)
+    params = attn_params(batch=B, num_heads=H, head_dim=d, n_max=n_max, total_tokens=T,
+                         max_seq_len=min(n_max, mc + microbatch), dtype=dt, alpha=alpha,
+                         num_ts_buckets=rab_ts.numel(), qkv_stride=qs, u_stride=us, ln_eps=ln_eps, flags=flags)
+    if num_splits is None:
+        num_splits = hstu_attn_paged_default_splits(
+            attn_params(batch=B, num_heads=H, head_dim=d, n_max=n_max, total_tokens=B * microbatch,
+                        max_seq_len=n_max, dtype=dt), mc)
+    if out is None:
+        out = torch.empty(T, H * d, dtype=dt, device=q_c.device)
+    hist_tokens = hist_timestamps.numel()
+    if workspace is None:
+        workspace = torch.empty(hstu_mfalcon_workspace_size(params, microbatch, num_splits, hist_tokens),
+                                dtype=torch.uint8, device=q_c.device)
+    rc = _lib.load().hstu_mfalcon_fwd(
+        ctypes.byref(params), _p(q_c), _p(k_c), _p(v_c), _p(u_c), _p(cand_offsets), _p(hist_timestamps),
+        _p(hist_ts_offsets), hist_tokens, _p(cand_timestamps), _p(rab_pos), _p(rab_ts), _p(ln_gamma), _p(ln_beta),
+        _p(k_pool), _p(v_pool), num_pages, _p(kv_page_table), kv_page_table.shape[1], page_size, _p(cached_lens),
+        max_candidates, microbatch, num_splits, _p(out), _p(workspace), workspace.numel(), _stream(stream))
+    _lib.check(rc, "hstu_mfalcon_fwd")
+    return out, workspace

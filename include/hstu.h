@@ -254,6 +254,42 @@ int hstu_layer_f1(const hstu_linear_params* p, const void* x, const void* w1, co
 int hstu_layer_f2(const hstu_linear_params* p, const void* y, const void* w2, const float* b2, void* x_next,
                   void* workspace, size_t workspace_bytes, hstu_stream_t stream);
 
+/* ---- M-FALCON: a large candidate set against the cached history -----------
+ *
+ * ("HSTU Generative Recommenders: Deploy on GPU Cloud", M-FALCON section:
+ * candidates are scored in microbatches in one pass over the shared history,
+ * the mask and relative bias modified so that each candidate sees the history
+ * and itself only.)  Candidate i of user u attends to the user's cached
+ * history (positions 0 .. L_u-1, read through the paged pool) and to itself;
+ * all of a user's candidates sit at position L_u.  Candidates never see one
+ * another, so the split into microbatches does not change any output.
+ *
+ * Each microbatch takes `microbatch` candidates of every user (users with
+ * fewer left are padded with zero rows whose outputs are dropped) and runs
+ * the paged forward once: microbatch + L_u must not exceed n_max.
+ *   q_c, k_c, v_c [T_c, H, d], u_c [T_c, H*d] dtype: candidates, user after
+ *                 user by cand_offsets [B+1] (p->total_tokens = T_c);
+ *                 row strides p->qkv_stride / p->u_stride as in hstu_attn_fwd
+ *   hist_timestamps [hist_tokens] int64, jagged by hist_ts_offsets [B+1]:
+ *                 each user's cached_lens[u] history timestamps
+ *   cand_timestamps [T_c] int64, non-decreasing per user and not before the
+ *                 user's last history timestamp
+ *   pool, page table, cached_lens as in hstu_attn_fwd_paged
+ *   max_candidates  host bound of candidates per user (sets the microbatch count)
+ *   out [T_c, H*d] dtype
+ * Device errors of any microbatch stay in the workspace's status word.
+ */
+size_t hstu_mfalcon_workspace_size(const hstu_attn_params* p, int32_t microbatch, int32_t num_splits,
+                                   int64_t hist_tokens);
+int hstu_mfalcon_fwd(const hstu_attn_params* p, const void* q_c, const void* k_c, const void* v_c,
+                     const void* u_c, const int32_t* cand_offsets, const int64_t* hist_timestamps,
+                     const int32_t* hist_ts_offsets, int64_t hist_tokens, const int64_t* cand_timestamps,
+                     const float* rab_pos, const float* rab_ts, const float* ln_gamma, const float* ln_beta,
+                     const void* k_pool, const void* v_pool, int32_t num_pages, const int32_t* kv_page_table,
+                     int32_t max_pages_per_user, int32_t page_size, const int32_t* cached_lens,
+                     int32_t max_candidates, int32_t microbatch, int32_t num_splits, void* out, void* workspace,
+                     size_t workspace_bytes, hstu_stream_t stream);
+
 /* ---- Paged KV cache: the write side --------------------------------------
  *
  * ("Recomendador generativo HSTU com Dynamo-Triton", KV cache section: the

@@ -179,3 +179,17 @@ def test_kv_rejects_bad_args_on_host(lib):
     assert lib.hstu_kv_append(ctypes.byref(kvp()), *([a] * 11), 16, None) == -5
     assert lib.hstu_kv_evict(ctypes.byref(kvp()), None, a, a, a, a, a, ws, None) == -1
     assert lib.hstu_kv_evict(ctypes.byref(kvp()), *([a] * 6), 16, None) == -5
+
+
+def test_mfalcon_rejects_bad_args_on_host(lib):
+    p = params()
+    a = ctypes.c_void_p(0x1000)
+    ws = 1 << 30
+    full = [a] * 7
+    assert lib.hstu_mfalcon_workspace_size(ctypes.byref(p), 0, 1, 100) == 0
+    assert lib.hstu_mfalcon_workspace_size(ctypes.byref(p), 128, 1, 100) > 0
+    args = lambda mb=128, q=a: ([ctypes.byref(p), q] + full[1:] + [100, a] + [a] * 6 +
+                                [10, a, 4, 32, a, 256, mb, 1, a, a, ws, None])
+    assert lib.hstu_mfalcon_fwd(*args(mb=0)) == -1
+    assert lib.hstu_mfalcon_fwd(*args(q=None)) == -1
+    assert lib.hstu_mfalcon_fwd(*args(q=ctypes.c_void_p(0x1008))) == -3
