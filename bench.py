@@ -459,6 +459,111 @@ def run_glue_bench(args, device):
                          "traffic": None}}
 
 
+def run_mfalcon_bench(args, device):
+    """M-FALCON: 8 users with a cached history of U[2048,4096] tokens (32-token
+    pages) score 4,096 candidates each, 1,024 per microbatch."""
+    import generative_recommender_attention_jagged_b200 as hstu
+    rng = np.random.default_rng(1000 + 31)
+    B, C, mb = 8, 4096, 1024
+    cached = rng.integers(2048, 4096, size=B, endpoint=True)
+    n_max = 4096 + mb
+    pb = synth.paged_batch(cached, 0, C, 4, 128, n_max, rng=rng, poison=False)
+    hist, hist_off, cand = [], [0], []
+    for b in range(B):
+        L = int(pb.cached_lens[b])
+        t = pb.timestamps[pb.ts_offsets[b]:pb.ts_offsets[b + 1]]
+        hist.append(t[:L])
+        cand.append(t[L:])
+        hist_off.append(hist_off[-1] + L)
+    d = dict(q=to_dev(pb.q), k=to_dev(pb.k), v=to_dev(pb.v), u=to_dev(pb.u),
+             off=to_dev(pb.new_offsets, torch.int32), hist=to_dev(np.concatenate(hist), torch.int64),
+             hoff=to_dev(np.array(hist_off), torch.int32), cts=to_dev(np.concatenate(cand), torch.int64),
+             rp=to_dev(pb.rab_pos, torch.float32), rt=to_dev(pb.rab_ts, torch.float32), kp=to_dev(pb.k_pool),
+             vp=to_dev(pb.v_pool), pt=to_dev(pb.kv_page_table, torch.int32), cl=to_dev(pb.cached_lens, torch.int32))
+    out, ws = None, None
+
+    def call():
+        nonlocal out, ws
+        out, ws = hstu.hstu_mfalcon_fwd(d["q"], d["k"], d["v"], d["u"], d["off"], d["hist"], d["hoff"], d["cts"],
+                                        d["rp"], d["rt"], d["kp"], d["vp"], d["pt"], d["cl"], n_max=n_max,
+                                        microbatch=mb, max_candidates=C, max_cached_len=int(cached.max()),
+                                        out=out, workspace=ws)
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 20))
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    if hstu.hstu_check_device_error(ws) != 0:
+        raise RuntimeError("mfalcon device status")
+    ms = a.elapsed_time(b) / steps
+    flops = float(sum(C * (int(L) + 1) for L in cached)) * 4 * 2 * (128 + 128)
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks, kind = measured_peaks()
+    peak = float(peaks["bf16_tflops_sustained"])
+    return {"workload": f"M-FALCON: B={B} users, cached history U[2048,4096] (32-token pages), {C} candidates "
+                        f"per user in microbatches of {mb}, H=4, d=128, bf16",
+            "ms": round(ms, 4), "candidates_per_s": round(B * C / (ms * 1e-3), 1), "tflops": round(tf, 1),
+            "roofline": {"kernel": "attn_sm100_kernel (paged, candidates)", "bound": "tensor",
+                         "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+                         "peak_source": f"{kind} bf16_tflops_sustained", "traffic": None}}
+
+
+def run_kv_append_bench(args, device):
+    """KV write side after a request of the paged workload: 8 users append 64
+    actions each (K and V, 4 heads x 128 bf16) into free pages."""
+    import generative_recommender_attention_jagged_b200 as hstu
+    rng = np.random.default_rng(1000 + 32)
+    B, A, P, H, D = 8, 64, 32, 4, 128
+    cached = rng.integers(6144, 8192, size=B, endpoint=True)
+    max_pages = int((cached.max() + A * 64) // P + 2)
+    num_pages = int(sum((c + A * 64) // P + 2 for c in cached))
+    k_pool = torch.zeros(num_pages, H, P, D, dtype=torch.bfloat16, device=device)
+    v_pool = torch.zeros_like(k_pool)
+    k_new = torch.randn(B * A, H, D, device=device).to(torch.bfloat16)
+    v_new = torch.randn(B * A, H, D, device=device).to(torch.bfloat16)
+    off = torch.arange(0, B * A + 1, A, dtype=torch.int32, device=device)
+    steps = max(3, min(args.steps, 50))
+
+    def fresh():
+        table = torch.full((B, max_pages), -1, dtype=torch.int32, device=device)
+        pages = [(int(c) + P - 1) // P for c in cached]
+        perm = torch.randperm(num_pages, device=device).to(torch.int32)
+        pos = 0
+        for b in range(B):
+            table[b, :pages[b]] = perm[pos:pos + pages[b]]
+            pos += pages[b]
+        free = perm[pos:].clone()
+        free = torch.cat([free, torch.zeros(pos, dtype=torch.int32, device=device)])
+        return table, torch.tensor(cached, dtype=torch.int32, device=device), free, \
+            torch.tensor([num_pages - pos], dtype=torch.int32, device=device)
+
+    table, lens, free, fc = fresh()
+    ws = hstu.hstu_kv_append(k_new, v_new, off, k_pool, v_pool, table, lens, free, fc)
+    torch.cuda.synchronize()
+    table, lens, free, fc = fresh()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):   # each call appends one more request's actions to every user
+        hstu.hstu_kv_append(k_new, v_new, off, k_pool, v_pool, table, lens, free, fc, workspace=ws)
+    b.record(stream)
+    torch.cuda.synchronize()
+    if hstu.hstu_check_device_error(ws) != 0:
+        raise RuntimeError("kv append device status")
+    us = a.elapsed_time(b) / steps * 1e3
+    moved = 2 * B * A * H * D * 2 * 2          # K and V, read + write
+    return {"workload": f"KV append: {B} users x {A} actions, H={H}, d={D}, bf16, {P}-token pages",
+            "us_per_call": round(us, 2), "bytes_per_call": moved,
+            "gbs": round(moved / (us * 1e-6) / 1e9, 1),
+            "note": "two launches (plan + copy) per call; at this size the call is launch-bound"}
+
+
 # ----------------------------------------------------------------------------
 # reference arm: the fp64 CPU oracle on the host cores
 # ----------------------------------------------------------------------------
@@ -502,6 +607,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-paged", action="store_true")
     ap.add_argument("--no-glue", action="store_true", help="skip the f1/f2 layer-glue timing")
+    ap.add_argument("--no-next", action="store_true", help="skip the M-FALCON and KV-append timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--paged-only", action="store_true",
                     help="run only the paged incremental sub-benchmark (profiling captures)")
@@ -536,6 +642,9 @@ def main():
         result["paged"] = run_paged_bench(args, device)
     if rank == 0 and not args.no_glue and world == 1:
         result["glue"] = run_glue_bench(args, device)
+    if rank == 0 and not args.no_next and world == 1:
+        result["mfalcon"] = run_mfalcon_bench(args, device)
+        result["kv_append"] = run_kv_append_bench(args, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
