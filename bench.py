@@ -169,11 +169,32 @@ def to_dev(x, dtype=None, device="cuda"):
     return x.to(device=device, dtype=dtype) if dtype is not None else x.to(device)
 
 
+def rank_seed(rank: int):
+    """Seed of a rank's users: rank 0 draws the workload's own users, every other
+    rank a distinct set (weak scaling: the same amount of work per rank)."""
+    return None if rank == 0 else 1000 + 7919 * rank
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its own, all get the max."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job(flops_per_rank_step: float, tokens_per_rank_step: float, world: int, ms_step: float):
+    """Whole-job throughput: all ranks' work over the slowest rank's step time."""
+    return (flops_per_rank_step * world / (ms_step * 1e-3) / 1e12,
+            tokens_per_rank_step * world / (ms_step * 1e-3))
+
+
 def run_ours(args, rank, world, device):
     import generative_recommender_attention_jagged_b200 as hstu
     from generative_recommender_attention_jagged_b200 import _lib
 
-    seed = None if rank == 0 else 1000 + 7919 * rank  # every rank its own users
+    seed = rank_seed(rank)  # every rank its own users
     layers = synth.attention_stack(args.workload, num_layers=args.layers, seed=seed)
     L = len(layers)
     b0 = layers[0]
@@ -233,18 +254,14 @@ def run_ours(args, rank, world, device):
     clk = clocks.stop()
     total_ms = t0.elapsed_time(t1)
     attn_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        tt = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, world, device)
 
     lengths = b0.lengths
     pairs = allowed_pairs(lengths, b0.num_candidates)
     flops_layer = pairs * H * FLOPS_PER_PAIR_HEAD
     flops_step = flops_layer * L
     ms_step = total_ms / args.steps
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
-    tokens_s = T * L * world / (ms_step * 1e-3)
+    value, tokens_s = whole_job(flops_step, T * L, world, ms_step)
     attn_avg_ms = float(np.mean(attn_ms))
     achieved = flops_layer / (attn_avg_ms * 1e-3) / 1e12
     tiles = issued_tiles(lengths, b0.num_candidates) * H
@@ -296,13 +313,9 @@ def run_ours(args, rank, world, device):
             e2e_step(True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=device, dtype=torch.float64)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
         e_step = e_ms / args.e2e_steps
-        e2e = {"value": round(flops_step * world / (e_step * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        e2e = {"value": round(whole_job(flops_step, T * L, world, e_step)[0], 3), "unit": "TFLOP/s",
                "ms_per_step": round(e_step, 3), "steps": args.e2e_steps,
                "h2d_bytes_per_step": h2d // args.e2e_steps, "d2h_bytes_per_step": d2h // args.e2e_steps}
 
