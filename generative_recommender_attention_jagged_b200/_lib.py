@@ -30,6 +30,7 @@ F_STAGE_ATTN = 0x20
 F_STAGE_EPILOGUE = 0x40
 
 LIN_SILU = 0x1
+LIN_CUBLAS = 0x2
 
 
 class AttnParams(ctypes.Structure):

@@ -206,11 +206,13 @@ def hstu_attn_fwd_static_ws(q, k, v, u, seq_offsets, timestamps, rab_pos, rab_ts
     return out
 
 
-def linear_params(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor, silu: bool) -> _lib.LinearParams:
+def linear_params(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor, silu: bool,
+                  force_cublas: bool = False) -> _lib.LinearParams:
     return _lib.LinearParams(rows=x.shape[0], d_in=x.shape[1], d_out=w.shape[1],
                              x_stride=x.stride(0) if x.shape[0] > 1 else x.shape[1],
                              out_stride=out.stride(0) if out.shape[0] > 1 else out.shape[1],
-                             dtype=_DT[x.dtype], flags=_lib.LIN_SILU if silu else 0)
+                             dtype=_DT[x.dtype],
+                             flags=(_lib.LIN_SILU if silu else 0) | (_lib.LIN_CUBLAS if force_cublas else 0))
 
 
 def hstu_linear_workspace_size(p: Optional[_lib.LinearParams] = None) -> int:
@@ -218,7 +220,7 @@ def hstu_linear_workspace_size(p: Optional[_lib.LinearParams] = None) -> int:
     return int(_lib.load().hstu_linear_workspace_size(ctypes.byref(p)))
 
 
-def _linear(name: str, x, w, bias, out, workspace, stream, silu: bool):
+def _linear(name: str, x, w, bias, out, workspace, stream, silu: bool, force_cublas: bool = False):
     for nm, t in (("x", x), ("w", w), ("out", out)):
         _need_cuda(nm, t, x.dtype)
     _need_cuda("bias", bias, torch.float32)
@@ -230,7 +232,7 @@ def _linear(name: str, x, w, bias, out, workspace, stream, silu: bool):
         out = torch.empty(x.shape[0], w.shape[1], dtype=x.dtype, device=x.device)
     if out.dim() != 2 or out.shape != (x.shape[0], w.shape[1]) or out.stride(1) != 1:
         raise ValueError(f"{name}: out [T, d_out] with contiguous rows expected")
-    p = linear_params(x, w, out, silu)
+    p = linear_params(x, w, out, silu, force_cublas)
     if workspace is None:
         workspace = torch.empty(hstu_linear_workspace_size(p), dtype=torch.uint8, device=x.device)
     rc = getattr(_lib.load(), name)(ctypes.byref(p), _p(x), _p(w), _p(bias), _p(out), _p(workspace),
@@ -239,19 +241,20 @@ def _linear(name: str, x, w, bias, out, workspace, stream, silu: bool):
     return out
 
 
-def hstu_layer_f1(x, w1, b1=None, *, out=None, workspace=None, stream=None):
+def hstu_layer_f1(x, w1, b1=None, *, out=None, workspace=None, stream=None, force_cublas: bool = False):
     """[U | V | Q | K] = SiLU(x W1 + b1) as one [T, 4*H*d] tensor (blocks head-major)."""
-    return _linear("hstu_layer_f1", x, w1, b1, out, workspace, stream, True)
+    return _linear("hstu_layer_f1", x, w1, b1, out, workspace, stream, True, force_cublas)
 
 
-def hstu_layer_f2(y, w2, b2=None, *, out=None, workspace=None, stream=None):
+def hstu_layer_f2(y, w2, b2=None, *, out=None, workspace=None, stream=None, force_cublas: bool = False):
     """x_next = y W2 + b2."""
-    return _linear("hstu_layer_f2", y, w2, b2, out, workspace, stream, False)
+    return _linear("hstu_layer_f2", y, w2, b2, out, workspace, stream, False, force_cublas)
 
 
-def hstu_linear(x, w, bias=None, *, silu: bool = False, out=None, workspace=None, stream=None):
+def hstu_linear(x, w, bias=None, *, silu: bool = False, out=None, workspace=None, stream=None,
+                force_cublas: bool = False):
     """out = act(x W + bias), act = SiLU or identity."""
-    return _linear("hstu_linear", x, w, bias, out, workspace, stream, silu)
+    return _linear("hstu_linear", x, w, bias, out, workspace, stream, silu, force_cublas)
 
 
 def split_uvqk(uvqk: torch.Tensor, num_heads: int, head_dim: int):

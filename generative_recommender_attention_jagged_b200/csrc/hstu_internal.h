@@ -25,6 +25,13 @@ struct BucketTable {
   unsigned int oct[32][4];
 };
 
+// Layer glue GEMM on the tensor cores (gemm_sm100.cu): out = act(x W + bias),
+// bf16, K a multiple of 64, N a multiple of 256; hdr = a workspace status header.
+bool gemm_sm100_supported(int K, int N);
+cudaError_t launch_gemm_sm100(const void* x, long long T, int K, long long x_stride, const void* w, int N,
+                              const float* bias, void* out, long long out_stride, bool silu, void* hdr,
+                              cudaStream_t s);
+
 // Built once per process in exact binary128 arithmetic (ts_table.cpp).
 const BucketTable& bucket_table(int num_buckets);
 

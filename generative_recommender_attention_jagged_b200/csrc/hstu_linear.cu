@@ -20,10 +20,12 @@
 #include <tuple>
 
 #include "hstu.h"
+#include "hstu_internal.h"
 
 namespace {
 
 constexpr size_t kLinearWorkspace = 32u << 20;  // cuBLASLt scratch for large-N GEMMs on sm_100
+constexpr size_t kHeaderBytes = 256;             // status word of the library's own GEMM
 
 // ---- SiLU in place ----------------------------------------------------------
 __device__ __forceinline__ float silu_f(float x) { return x / (1.f + __expf(-x)); }
@@ -165,16 +167,28 @@ int enqueue_gemm(int dev, const hstu_linear_params& p, long long xs, long long o
   return rc;
 }
 
-// cuBLASLt scratch, then (bf16) the bias converted to bf16
+// status header, cuBLASLt scratch, then (bf16) the bias converted to bf16
 size_t workspace_bytes(const hstu_linear_params& p) {
-  return kLinearWorkspace + (p.d_out > 0 ? ((size_t)p.d_out * 2 + 255) / 256 * 256 : 0);
+  return kHeaderBytes + kLinearWorkspace + (p.d_out > 0 ? ((size_t)p.d_out * 2 + 255) / 256 * 256 : 0);
+}
+
+bool device_is_sm100(int dev) {
+  static int cached[64];  // 0 unknown, 1 yes, 2 no
+  if (dev < 0 || dev >= 64) return false;
+  if (cached[dev] == 0) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return cached[dev] == 1;
 }
 
 int run_linear(const hstu_linear_params* p, const void* x, const void* w, const float* bias, void* out,
                void* ws, size_t ws_bytes, cudaStream_t stream, bool silu) {
   if (!p || p->rows < 0 || p->d_in <= 0 || p->d_out <= 0) return HSTU_ERR_INVALID_ARG;
   if (p->dtype != HSTU_DT_BF16 && p->dtype != HSTU_DT_F32) return HSTU_ERR_INVALID_ARG;
-  if (p->flags & ~HSTU_LIN_SILU) return HSTU_ERR_INVALID_ARG;
+  if (p->flags & ~(HSTU_LIN_SILU | HSTU_LIN_CUBLAS)) return HSTU_ERR_INVALID_ARG;
   const long long xs = p->x_stride ? p->x_stride : p->d_in;
   const long long os = p->out_stride ? p->out_stride : p->d_out;
   if (xs < p->d_in || os < p->d_out) return HSTU_ERR_INVALID_ARG;
@@ -186,6 +200,19 @@ int run_linear(const hstu_linear_params* p, const void* x, const void* w, const 
   if (ws_bytes < workspace_bytes(*p)) return HSTU_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
+  char* wsc = static_cast<char*>(ws);
+  // the library's GEMM where its fused epilogue pays: with SiLU (no second pass over
+  // the output) or wide outputs; narrow plain GEMMs (f2) are faster on cuBLASLt
+  if (p->dtype == HSTU_DT_BF16 && !(p->flags & HSTU_LIN_CUBLAS) && device_is_sm100(dev) &&
+      hstu::gemm_sm100_supported(p->d_in, p->d_out) && (silu || p->d_out >= 1024)) {
+    // the library's own GEMM: bias and activation in its epilogue
+    if (cudaMemsetAsync(wsc, 0, kHeaderBytes, stream) != cudaSuccess) return HSTU_ERR_CUDA;
+    return hstu::launch_gemm_sm100(x, p->rows, p->d_in, xs, w, p->d_out, bias, out, os, silu, wsc, stream) ==
+                   cudaSuccess
+               ? HSTU_OK
+               : HSTU_ERR_CUDA;
+  }
+  ws = wsc + kHeaderBytes;
   const void* gemm_bias = bias;
   if (bias && p->dtype == HSTU_DT_BF16) {
     __nv_bfloat16* b16 = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + kLinearWorkspace);

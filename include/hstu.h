@@ -214,12 +214,17 @@ int hstu_ts_bucket(const int64_t* dt, int64_t n, int32_t num_buckets, int32_t* o
  * the four blocks of one [T, 4*H*d] buffer are directly the u, v, q, k
  * arguments of hstu_attn_fwd (token stride 4*H*d).
  *
- * Both are plain GEMMs (cuBLASLt, fp32 accumulate, bias added in the GEMM
- * epilogue); f1's SiLU runs in place right after it in one vectorised kernel.
- * The first call on a device creates that device's cuBLASLt handle (host
- * memory owned by cuBLASLt); nothing else is allocated.
+ * bf16 calls with d_in a multiple of 64, d_out a multiple of 256 and either
+ * SiLU (f1) or d_out >= 1024 run the library's own tcgen05 GEMM with the fp32
+ * bias and the SiLU in its epilogue (one pass over the output).  Other calls
+ * (f2's narrow 512-column output, fp32, HSTU_LIN_CUBLAS) use cuBLASLt (fp32 accumulate, bias in its epilogue) and,
+ * for f1, an in-place SiLU kernel.  The first cuBLASLt call on a device
+ * creates that device's handle (host memory owned by cuBLASLt); nothing else
+ * is allocated.  The workspace begins with a status word
+ * (hstu_check_device_error) that reports a timed-out wait of the GEMM.
  */
-#define HSTU_LIN_SILU 0x1u  /* hstu_linear only: apply SiLU to the output (f1) */
+#define HSTU_LIN_SILU 0x1u    /* hstu_linear only: apply SiLU to the output (f1)             */
+#define HSTU_LIN_CUBLAS 0x2u  /* use the cuBLASLt GEMM even where the library's own applies  */
 
 typedef struct {
   int64_t rows;        /* T (0 is allowed: nothing to do)                              */
@@ -228,11 +233,11 @@ typedef struct {
   int64_t x_stride;    /* elements between rows of x; 0 = d_in; a multiple of 8        */
   int64_t out_stride;  /* elements between rows of out; 0 = d_out; a multiple of 8     */
   hstu_dtype dtype;    /* x, w, out: bf16 (fp32 accumulate) or fp32                     */
-  uint32_t flags;      /* HSTU_LIN_SILU or 0                                            */
+  uint32_t flags;      /* HSTU_LIN_SILU, HSTU_LIN_CUBLAS                                */
 } hstu_linear_params;
 
-/* Bytes of workspace the linear entry points use: cuBLASLt scratch (32 MiB)
- * plus room for the bf16 copy of the bias. */
+/* Bytes of workspace the linear entry points use: a 256-byte status header,
+ * cuBLASLt scratch (32 MiB) and room for a bf16 copy of the bias. */
 size_t hstu_linear_workspace_size(const hstu_linear_params* p);
 
 /* out[r, :] = act(x[r, :] W + bias), act = SiLU with HSTU_LIN_SILU, else identity.

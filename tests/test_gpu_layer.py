@@ -106,3 +106,37 @@ def test_whole_layer_matches_oracle():
     want = olayer.layer(host64(s.x), host64(w1), w.b1, host64(w2), w.b2, s.seq_offsets, s.timestamps, None,
                         rab_pos, rab_ts, s.alpha, s.n_max, H, D, rows=rows)
     assert rel_err(got[rows], want) <= BF16_TOL
+
+
+@pytest.mark.parametrize("T", [1, 300, 4099])
+def test_own_gemm_and_cublas_agree_with_the_oracle(T):
+    """bf16 f1 runs the library's tcgen05 GEMM (bias and SiLU in its epilogue),
+    and so does any wide plain GEMM; the cuBLASLt path must agree within the
+    bf16 tolerance."""
+    w1, b1, w2, b2 = weights(T + 7)
+    x = dev(x_rows(T, T + 7))
+    z_own = hstu.hstu_layer_f1(x, dev(w1), dev(b1))
+    z_lib = hstu.hstu_layer_f1(x, dev(w1), dev(b1), force_cublas=True)
+    y_own = hstu.hstu_layer_f2(z_own[:, :DM].contiguous(), dev(w2), dev(b2))
+    y_lib = hstu.hstu_layer_f2(z_own[:, :DM].contiguous(), dev(w2), dev(b2), force_cublas=True)
+    torch.cuda.synchronize()
+    u, v, q, k = olayer.f1(host64(x), host64(w1), b1, H, D)
+    want = np.concatenate([u, v.reshape(T, -1), q.reshape(T, -1), k.reshape(T, -1)], axis=1)
+    assert rel_err(host64(z_own), want) <= BF16_TOL
+    assert rel_err(host64(z_lib), want) <= BF16_TOL
+    y_want = olayer.f2(host64(z_own[:, :DM]), host64(w2), b2)
+    assert rel_err(host64(y_own), y_want) <= BF16_TOL
+    assert rel_err(host64(y_lib), y_want) <= BF16_TOL
+    assert not torch.equal(z_own, z_lib) or T == 1   # two different kernels ran
+
+
+def test_own_gemm_plain_wide_output():
+    T = 777
+    w1, b1, _, _ = weights(21)
+    x = dev(x_rows(T, 21))
+    own = hstu.hstu_linear(x, dev(w1), dev(b1))               # 2048 columns, no activation
+    lib = hstu.hstu_linear(x, dev(w1), dev(b1), force_cublas=True)
+    torch.cuda.synchronize()
+    want = host64(x) @ host64(w1) + b1
+    assert rel_err(host64(own), want) <= BF16_TOL and rel_err(host64(lib), want) <= BF16_TOL
+    assert not torch.equal(own, lib)
