@@ -632,6 +632,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--paged-only", action="store_true",
                     help="run only the paged incremental sub-benchmark (profiling captures)")
+    ap.add_argument("--glue-only", action="store_true", help="run only the f1/f2 timing (profiling captures)")
+    ap.add_argument("--next-only", action="store_true",
+                    help="run only the M-FALCON and KV-append timings (profiling captures)")
     ap.add_argument("--layers", type=int, default=None,
                     help="fewer layers (profiling captures only; the bench line uses all 8)")
     args = ap.parse_args()
@@ -657,6 +660,15 @@ def main():
     if args.paged_only:
         if rank == 0:
             print(json.dumps({"paged": run_paged_bench(args, device)}), flush=True)
+        return
+    if args.glue_only:
+        if rank == 0:
+            print(json.dumps({"glue": run_glue_bench(args, device)}), flush=True)
+        return
+    if args.next_only:
+        if rank == 0:
+            print(json.dumps({"mfalcon": run_mfalcon_bench(args, device),
+                              "kv_append": run_kv_append_bench(args, device)}), flush=True)
         return
     result, b0 = run_ours(args, rank, world, device)
     if rank == 0 and not args.no_paged and world == 1:
