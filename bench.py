@@ -482,10 +482,10 @@ def run_glue_bench(args, device):
 
 def run_mfalcon_bench(args, device):
     """M-FALCON: 8 users with a cached history of U[2048,4096] tokens (32-token
-    pages) score 4,096 candidates each, 1,024 per microbatch."""
+    pages) score 4,096 candidates each, 2,048 per microbatch."""
     import generative_recommender_attention_jagged_b200 as hstu
     rng = np.random.default_rng(1000 + 31)
-    B, C, mb = 8, 4096, 1024
+    B, C, mb = 8, 4096, 2048
     cached = rng.integers(2048, 4096, size=B, endpoint=True)
     n_max = 4096 + mb
     pb = synth.paged_batch(cached, 0, C, 4, 128, n_max, rng=rng, poison=False)

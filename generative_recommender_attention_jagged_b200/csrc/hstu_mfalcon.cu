@@ -251,10 +251,13 @@ int hstu_mfalcon_fwd(const hstu_attn_params* p, const void* q_c, const void* k_c
   mf_meta_kernel<<<1, 1024, 0, s>>>(a);
   if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
   const int n_mb = (max_candidates + microbatch - 1) / microbatch;
-  const int gy = std::max(1, std::min(16, (int)((4ll * microbatch * hd * esize / 16 + 4095) / 4096)));
+  // enough blocks per user that each thread moves about four 16-byte pieces
+  const long long row_chunks = hd * esize / 16;
+  const int gy_gather = (int)std::max(1ll, std::min(256ll, (4ll * microbatch * row_chunks + 1023) / 1024));
+  const int gy_scatter = (int)std::max(1ll, std::min(256ll, ((long long)microbatch * row_chunks + 1023) / 1024));
   for (int m = 0; m < n_mb; ++m) {
     a.m = m;
-    mf_gather_kernel<<<dim3(p->batch, gy), 256, 0, s>>>(a);
+    mf_gather_kernel<<<dim3(p->batch, gy_gather), 256, 0, s>>>(a);
     if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
     const int rc = hstu_attn_fwd_paged(&pp, a.q_mb, a.k_mb, a.v_mb, a.u_mb, a.new_off, a.ts_mb, a.ts_off, a.ncand,
                                        rab_pos, rab_ts, ln_gamma, ln_beta, k_pool, v_pool, num_pages,
@@ -263,7 +266,7 @@ int hstu_mfalcon_fwd(const hstu_attn_params* p, const void* q_c, const void* k_c
     if (rc != HSTU_OK) return rc;
     mf_status_kernel<<<1, 32, 0, s>>>(reinterpret_cast<WsHeader*>(ws),
                                       reinterpret_cast<const WsHeader*>(ws + l.paged_off));
-    mf_scatter_kernel<<<dim3(p->batch, gy), 256, 0, s>>>(a);
+    mf_scatter_kernel<<<dim3(p->batch, gy_scatter), 256, 0, s>>>(a);
     if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
   }
   return HSTU_OK;
