@@ -69,6 +69,16 @@ def issued_tiles(lengths, cands=None):
     return tiles
 
 
+def max_sm_mhz(device_index: int = 0) -> int:
+    """clocks.max.sm from nvidia-smi (1965 MHz on this part if it cannot be read)."""
+    try:
+        out = subprocess.run(["nvidia-smi", "-i", str(device_index), "--query-gpu=clocks.max.sm",
+                              "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+        return int(out.stdout.strip().splitlines()[0])
+    except Exception:
+        return 1965
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
 
@@ -535,6 +545,46 @@ def run_mfalcon_bench(args, device):
                          "peak_source": f"{kind} bf16_tflops_sustained", "traffic": None}}
 
 
+def run_bwd_bench(args, device):
+    """Backward of the attention core (CUDA cores, fp32) on one layer of the
+    32-user layer workload: d_q, d_k, d_v and the bias-table gradients."""
+    import generative_recommender_attention_jagged_b200 as hstu
+    b = synth.workload_attention("layer_bf16", layer=0)
+    T, H, d = b.q.shape
+    g = torch.randn(T, H, d, device=device)
+    x = dict(q=to_dev(b.q), k=to_dev(b.k), v=to_dev(b.v), off=to_dev(b.seq_offsets, torch.int32),
+             ts=to_dev(b.timestamps, torch.int64), rp=to_dev(b.rab_pos, torch.float32),
+             rt=to_dev(b.rab_ts, torch.float32))
+
+    def call():
+        return hstu.hstu_attn_bwd(x["q"], x["k"], x["v"], x["off"], x["ts"], x["rp"], x["rt"], g, n_max=b.n_max,
+                                  alpha=b.alpha, max_seq_len=b.max_seq_len)
+    out = call()
+    torch.cuda.synchronize()
+    if hstu.hstu_check_device_error(out[-1]) != 0:
+        raise RuntimeError("backward device status")
+    steps = max(3, min(args.steps, 5))
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    pairs = allowed_pairs(b.lengths, b.num_candidates)
+    flops = pairs * H * 4 * 2 * d          # d_v, d_a, d_q, d_k: four products of 2 d flops per pair
+    tf = flops / (ms * 1e-3) / 1e12
+    clk = max_sm_mhz()
+    peak = 148 * 128 * 2 * clk * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
+    return {"workload": f"layer_bf16 backward: B={b.batch} users, lengths U[512,1024] (T={T}), H={H}, d={d}, "
+                        f"fp32 on CUDA cores", "ms": round(ms, 3), "tflops": round(tf, 2),
+            "roofline": {"kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel", "bound": "alu",
+                         "achieved": round(tf, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                         "frac": round(tf / peak, 4),
+                         "peak_source": f"148 SMs x 128 fp32 FMA lanes x 2 flops x {clk} MHz", "traffic": None}}
+
+
 def run_kv_append_bench(args, device):
     """KV write side after a request of the paged workload: 8 users append 64
     actions each (K and V, 4 heads x 128 bf16) into free pages."""
@@ -668,7 +718,8 @@ def main():
     if args.next_only:
         if rank == 0:
             print(json.dumps({"mfalcon": run_mfalcon_bench(args, device),
-                              "kv_append": run_kv_append_bench(args, device)}), flush=True)
+                              "kv_append": run_kv_append_bench(args, device),
+                              "backward": run_bwd_bench(args, device)}), flush=True)
         return
     result, b0 = run_ours(args, rank, world, device)
     if rank == 0 and not args.no_paged and world == 1:
@@ -678,6 +729,7 @@ def main():
     if rank == 0 and not args.no_next and world == 1:
         result["mfalcon"] = run_mfalcon_bench(args, device)
         result["kv_append"] = run_kv_append_bench(args, device)
+        result["backward"] = run_bwd_bench(args, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()

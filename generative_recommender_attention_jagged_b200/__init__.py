@@ -9,6 +9,7 @@ through its C ABI (include/hstu.h).  This package is the thin Python binding.
 from ._lib import AttnParams, HstuError, LIB_PATH  # noqa: F401
 from .api import (  # noqa: F401
     attn_params,
+    hstu_attn_bwd,
     hstu_attn_fwd,
     hstu_attn_fwd_paged,
     hstu_attn_paged_default_splits,
@@ -36,5 +37,5 @@ __all__ = [
     "hstu_check_device_error", "hstu_status_string", "hstu_ts_bucket", "hstu_version",
     "hstu_layer_f1", "hstu_layer_f2", "hstu_linear", "hstu_linear_workspace_size", "split_uvqk",
     "hstu_kv_append", "hstu_kv_evict", "hstu_kv_workspace_size", "hstu_mfalcon_fwd",
-    "hstu_mfalcon_workspace_size",
+    "hstu_mfalcon_workspace_size", "hstu_attn_bwd",
 ]

@@ -121,6 +121,10 @@ def load() -> ctypes.CDLL:
         fn.restype = ctypes.c_int
     lib.hstu_attn_fwd_static_ws.argtypes = [PP] + [P] * 13
     lib.hstu_attn_fwd_static_ws.restype = ctypes.c_int
+    lib.hstu_attn_bwd_workspace_size.argtypes = [PP]
+    lib.hstu_attn_bwd_workspace_size.restype = sz
+    lib.hstu_attn_bwd.argtypes = [PP] + [P] * 15 + [sz, P]
+    lib.hstu_attn_bwd.restype = ctypes.c_int
     lib.hstu_mfalcon_workspace_size.argtypes = [PP, i32, i32, i64]
     lib.hstu_mfalcon_workspace_size.restype = sz
     lib.hstu_mfalcon_fwd.argtypes = ([PP] + [P] * 7 + [i64, P] + [P] * 6 + [i32, P, i32, i32, P, i32, i32, i32, P, P,

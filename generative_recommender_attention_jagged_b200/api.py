@@ -374,3 +374,40 @@ def hstu_mfalcon_fwd(q_c, k_c, v_c, u_c, cand_offsets, hist_timestamps, hist_ts_
         max_candidates, microbatch, num_splits, _p(out), _p(workspace), workspace.numel(), _stream(stream))
     _lib.check(rc, "hstu_mfalcon_fwd")
     return out, workspace
+
+
+def hstu_attn_bwd(q, k, v, seq_offsets, timestamps, rab_pos, rab_ts, d_o, *, n_max: int,
+                  alpha: Optional[float] = None, num_candidates=None, max_seq_len: Optional[int] = None,
+                  workspace=None, stream=None):
+    """Gradients of the raw per-head output o = A V: returns d_q, d_k, d_v [T, H, d]
+    and d_rab_pos, d_rab_ts (all fp32)."""
+    T, H, d = q.shape
+    dt = q.dtype
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, dt)
+    _need_cuda("d_o", d_o, torch.float32)
+    _need_cuda("seq_offsets", seq_offsets, torch.int32)
+    _need_cuda("timestamps", timestamps, torch.int64)
+    _need_cuda("num_candidates", num_candidates, torch.int32)
+    _need_cuda("rab_pos", rab_pos, torch.float32)
+    _need_cuda("rab_ts", rab_ts, torch.float32)
+    if not d_o.is_contiguous() or d_o.shape != q.shape:
+        raise ValueError("d_o must be a contiguous [T, H, d] tensor")
+    qs = _rows_view("q", q, H, d)
+    if _rows_view("k", k, H, d) != qs or _rows_view("v", v, H, d) != qs:
+        raise ValueError("q, k and v must share one token stride")
+    params = attn_params(batch=seq_offsets.numel() - 1, num_heads=H, head_dim=d, n_max=n_max, total_tokens=T,
+                         max_seq_len=n_max if max_seq_len is None else max_seq_len, dtype=dt, alpha=alpha,
+                         num_ts_buckets=rab_ts.numel(), qkv_stride=qs)
+    grads = [torch.empty(T, H, d, dtype=torch.float32, device=q.device) for _ in range(3)]
+    d_rp = torch.empty_like(rab_pos)
+    d_rt = torch.empty_like(rab_ts)
+    if workspace is None:
+        workspace = torch.empty(int(_lib.load().hstu_attn_bwd_workspace_size(ctypes.byref(params))),
+                                dtype=torch.uint8, device=q.device)
+    rc = _lib.load().hstu_attn_bwd(ctypes.byref(params), _p(q), _p(k), _p(v), _p(seq_offsets), _p(timestamps),
+                                   _p(num_candidates), _p(rab_pos), _p(rab_ts), _p(d_o), _p(grads[0]),
+                                   _p(grads[1]), _p(grads[2]), _p(d_rp), _p(d_rt), _p(workspace),
+                                   workspace.numel(), _stream(stream))
+    _lib.check(rc, "hstu_attn_bwd")
+    return grads[0], grads[1], grads[2], d_rp, d_rt, workspace

@@ -329,6 +329,59 @@ int hstu_attn_fwd_paged(const hstu_attn_params* p, const void* q_new, const void
   return run(p, c);
 }
 
+size_t hstu_attn_bwd_workspace_size(const hstu_attn_params* p) {
+  return check_params(p) == HSTU_OK ? sizeof(WsHeader) : 0;
+}
+
+int hstu_attn_bwd(const hstu_attn_params* p, const void* q, const void* k, const void* v,
+                  const int32_t* seq_offsets, const int64_t* timestamps, const int32_t* num_candidates,
+                  const float* rab_pos, const float* rab_ts, const float* d_o, float* d_q, float* d_k, float* d_v,
+                  float* d_rab_pos, float* d_rab_ts, void* workspace, size_t workspace_bytes,
+                  hstu_stream_t stream) {
+  if (int rc = check_params(p)) return rc;
+  if (!q || !k || !v || !seq_offsets || !timestamps || !rab_pos || !rab_ts || !d_o || !d_q || !d_k || !d_v ||
+      !d_rab_pos || !d_rab_ts || !workspace)
+    return HSTU_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, d_o, d_q, d_k, d_v, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return HSTU_ERR_ALIGNMENT;
+  if (workspace_bytes < sizeof(WsHeader)) return HSTU_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  AttnArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.B = p->batch;
+  a.H = p->num_heads;
+  a.d = p->head_dim;
+  a.n_max = p->n_max;
+  a.nb = p->num_ts_buckets;
+  a.T_q = p->total_tokens;
+  a.qkv_stride = p->qkv_stride ? p->qkv_stride : p->num_heads * p->head_dim;
+  a.u_stride = a.qkv_stride;
+  a.alpha = p->alpha;
+  a.num_splits = 1;
+  a.in_bf16 = p->dtype == HSTU_DT_BF16 ? 1 : 0;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.q_offsets = seq_offsets;
+  a.ts = timestamps;
+  a.ts_offsets = seq_offsets;
+  a.num_cand = num_candidates;
+  a.rab_pos = rab_pos;
+  a.rab_ts = rab_ts;
+  a.hdr = static_cast<WsHeader*>(workspace);
+  if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), s) != cudaSuccess ||
+      cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * (size_t)p->n_max - 1), s) != cudaSuccess ||
+      cudaMemsetAsync(d_rab_ts, 0, sizeof(float) * (size_t)p->num_ts_buckets, s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (a.T_q == 0) return HSTU_OK;
+  // the forward's checks of offsets, lengths, candidate counts and timestamps
+  if (launch_plan(a, false, p->max_seq_len, s) != cudaSuccess) return HSTU_ERR_CUDA;
+  const BucketTable& thr = bucket_table(a.nb);
+  return launch_attn_bwd(a, thr, d_o, d_q, d_k, d_v, d_rab_pos, d_rab_ts, s) == cudaSuccess ? HSTU_OK
+                                                                                            : HSTU_ERR_CUDA;
+}
+
 int hstu_ts_bucket(const int64_t* dt, int64_t n, int32_t num_buckets, int32_t* out, hstu_stream_t stream) {
   if (n < 0 || num_buckets <= 0 || num_buckets > kMaxBuckets) return HSTU_ERR_INVALID_ARG;
   if (n > 0 && (!dt || !out)) return HSTU_ERR_INVALID_ARG;

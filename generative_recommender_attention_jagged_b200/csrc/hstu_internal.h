@@ -118,6 +118,11 @@ cudaError_t launch_attn_sm100(const AttnArgs& a, const BucketTable& thr, const C
                               const CUtensorMap& tm_kpool, const CUtensorMap& tm_vpool,
                               cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnArgs& a, const BucketTable& thr, cudaStream_t s);
+
+// Backward of the attention core on CUDA cores (hstu_bwd.cu); gradients fp32,
+// d_rp / d_rt must be zeroed by the caller.
+cudaError_t launch_attn_bwd(const AttnArgs& a, const BucketTable& thr, const float* d_o, float* dq, float* dk,
+                            float* dv, float* d_rp, float* d_rt, cudaStream_t s);
 cudaError_t launch_epilogue(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_ts_bucket(const int64_t* dt, int64_t n, int32_t* out, const BucketTable& thr,
                              cudaStream_t s);

@@ -259,6 +259,32 @@ int hstu_layer_f1(const hstu_linear_params* p, const void* x, const void* w1, co
 int hstu_layer_f2(const hstu_linear_params* p, const void* y, const void* w2, const float* b2, void* x_next,
                   void* workspace, size_t workspace_bytes, hstu_stream_t stream);
 
+/* ---- Backward of the attention core ----------------------------------------
+ *
+ * For training ("How Generative Recommenders Are Redefining RecSys at Scale",
+ * Summary: the models are trained at scale): given d_o = dL/do for the raw
+ * per-head output o = A V (before the LayerNorm gate; the gate's backward is
+ * elementwise and not part of this call), the gradients of q, k, v and of the
+ * two bias tables over jagged users (no paged prefix):
+ *   ds_ij = (d_o_i . v_j) SiLU'(s_ij) / n_max on the allowed set,
+ *           SiLU'(x) = sig(x) (1 + x (1 - sig(x)))
+ *   d_q_i = alpha sum_j ds_ij k_j,   d_k_j = alpha sum_i ds_ij q_i,
+ *   d_v_j = sum_i a_ij d_o_i,        d_rab_pos[p(i)-p(j)+n_max-1] += ds_ij,
+ *   d_rab_ts[b(i,j)] += ds_ij
+ * Computed on CUDA cores in fp32 (scores recomputed as in the forward).
+ *   q, k, v     [T, H, d] dtype with token stride p->qkv_stride
+ *   d_o         [T, H, d] fp32 contiguous
+ *   d_q, d_k, d_v [T, H, d] fp32 contiguous (written)
+ *   d_rab_pos   [2*n_max-1] fp32, d_rab_ts [num_ts_buckets] fp32 (zeroed, then summed)
+ * Device checks as in hstu_attn_fwd (status word in the workspace).
+ */
+size_t hstu_attn_bwd_workspace_size(const hstu_attn_params* p);
+int hstu_attn_bwd(const hstu_attn_params* p, const void* q, const void* k, const void* v,
+                  const int32_t* seq_offsets, const int64_t* timestamps, const int32_t* num_candidates,
+                  const float* rab_pos, const float* rab_ts, const float* d_o, float* d_q, float* d_k, float* d_v,
+                  float* d_rab_pos, float* d_rab_ts, void* workspace, size_t workspace_bytes,
+                  hstu_stream_t stream);
+
 /* ---- M-FALCON: a large candidate set against the cached history -----------
  *
  * ("HSTU Generative Recommenders: Deploy on GPU Cloud", M-FALCON section:

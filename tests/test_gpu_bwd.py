@@ -1,0 +1,60 @@
+"""GPU backward of the attention core against the fp64 backward oracle
+(itself pinned by finite differences of the forward oracle)."""
+import numpy as np
+import pytest
+import torch
+
+import generative_recommender_attention_jagged_b200 as hstu
+import synth
+from oracle import backward as obwd
+
+from .gpu_helpers import dev, rel_err
+
+pytestmark = pytest.mark.gpu
+
+# The backward runs in fp32 on the same rounded inputs the oracle upcasts; a
+# gradient entry sums up to N_max terms, so fp32 rounding stays well below 1e-4
+# of the largest entry.
+BWD_TOL = 1e-4
+
+
+def run(b, seed):
+    rng = np.random.default_rng(seed)
+    g = rng.standard_normal(tuple(b.q.shape)).astype(np.float32)
+    dq, dk, dv, drp, drt, ws = hstu.hstu_attn_bwd(
+        dev(b.q), dev(b.k), dev(b.v), dev(b.seq_offsets, torch.int32), dev(b.timestamps, torch.int64),
+        dev(b.rab_pos, torch.float32), dev(b.rab_ts, torch.float32), dev(g), n_max=b.n_max, alpha=b.alpha,
+        num_candidates=dev(b.num_candidates, torch.int32), max_seq_len=b.max_seq_len)
+    status = hstu.hstu_check_device_error(ws)
+    want = obwd.attn_jagged_bwd(b.q, b.k, b.v, b.seq_offsets, b.timestamps, b.num_candidates, b.rab_pos,
+                                b.rab_ts, b.alpha, b.n_max, g)
+    got = [t.cpu().double().numpy() for t in (dq, dk, dv, drp, drt)]
+    return status, got, want
+
+
+@pytest.mark.parametrize("lengths,cands,H,d,dtype", [
+    ([37, 64], None, 2, 32, torch.float32),
+    ([50, 1, 77], [10, 0, 77], 2, 32, torch.float32),
+    ([300, 129], [40, 0], 4, 128, torch.bfloat16),
+])
+def test_gradients_match_oracle(lengths, cands, H, d, dtype):
+    rng = np.random.default_rng(sum(lengths))
+    b = synth.jagged_batch(lengths, H, d, 512, rng=rng, dtype=dtype, num_candidates=cands,
+                           qkvu_scale=1.0 / np.sqrt(d) if dtype == torch.float32 else 1.0)
+    status, got, want = run(b, seed=7)
+    assert status == 0
+    for name, gv, wv in zip(("d_q", "d_k", "d_v", "d_rab_pos", "d_rab_ts"), got, want):
+        assert rel_err(gv, wv) <= BWD_TOL, name
+
+
+def test_unsorted_timestamps_are_reported():
+    rng = np.random.default_rng(3)
+    b = synth.jagged_batch([20], 2, 32, 64, rng=rng, dtype=torch.float32)
+    b.timestamps = b.timestamps.copy()
+    b.timestamps[5] = b.timestamps[4] - 10
+    rng2 = np.random.default_rng(0)
+    g = rng2.standard_normal(tuple(b.q.shape)).astype(np.float32)
+    *_, ws = hstu.hstu_attn_bwd(dev(b.q), dev(b.k), dev(b.v), dev(b.seq_offsets, torch.int32),
+                                dev(b.timestamps, torch.int64), dev(b.rab_pos, torch.float32),
+                                dev(b.rab_ts, torch.float32), dev(g), n_max=b.n_max, alpha=b.alpha)
+    assert hstu.hstu_check_device_error(ws) == -8
