@@ -563,15 +563,19 @@ def run_bwd_bench(args, device):
     torch.cuda.synchronize()
     if hstu.hstu_check_device_error(out[-1]) != 0:
         raise RuntimeError("backward device status")
-    steps = max(3, min(args.steps, 5))
+    steps = max(5, min(args.steps, 20))
     stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
+    for _ in range(2):
         call()
-    e1.record(stream)
+    ev = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        ev.append((e0, e1))
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+    ms = float(np.median([x.elapsed_time(y) for x, y in ev]))   # per call, median
     pairs = allowed_pairs(b.lengths, b.num_candidates)
     flops = pairs * H * 4 * 2 * d          # d_v, d_a, d_q, d_k: four products of 2 d flops per pair
     tf = flops / (ms * 1e-3) / 1e12
@@ -579,7 +583,7 @@ def run_bwd_bench(args, device):
     peak = 148 * 128 * 2 * clk * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
     return {"workload": f"layer_bf16 backward: B={b.batch} users, lengths U[512,1024] (T={T}), H={H}, d={d}, "
                         f"fp32 on CUDA cores", "ms": round(ms, 3), "tflops": round(tf, 2),
-            "roofline": {"kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel", "bound": "alu",
+            "roofline": {"kernel": "attn_bwd_tiled_kernel", "bound": "alu",
                          "achieved": round(tf, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
                          "frac": round(tf / peak, 4),
                          "peak_source": f"148 SMs x 128 fp32 FMA lanes x 2 flops x {clk} MHz", "traffic": None}}

@@ -10,8 +10,19 @@
 //   dv_j  = sum_i a_ij g_i,  a_ij = SiLU(s_ij) / N_max
 //   dk_j  = alpha sum_i ds_ij q_i          (key-side kernel, one warp per (key, head))
 // Scores are recomputed in fp32 exactly as the CUDA-core forward does them
-// (exact integer time buckets, expf).  The bias gradients are summed with
-// atomics: a warp first folds runs of equal indices of its own row.
+// (exact integer time buckets, expf).
+//
+// Head dims 32, 64 and 128 take the tiled kernel: one CTA per (user, head,
+// block of 64 keys) keeps K, V and the block's d_k, d_v accumulators on chip
+// and walks the 64-row query blocks that see the keys.  Per query block it
+// stages Q and g in shared memory, forms S = Q K^T and dP = g V^T (4x4
+// register tiles, fp32 FMA), turns them into a and ds, then accumulates
+// d_v += a^T g and d_k += ds^T Q, and adds ds K into d_q with vector atomics
+// (d_q is zeroed first).  Bias gradients are folded per thread, summed in
+// shared memory (a 127-entry window of position differences per block pair, a
+// bucket histogram per CTA) and added to global memory with atomics.  Other
+// head dims take the warp-per-row kernels below, whose warps fold runs of
+// equal bias indices of their own row before the atomics.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -220,11 +231,328 @@ __global__ void __launch_bounds__(256) attn_bwd_kv_kernel(const AttnArgs a, cons
   }
 }
 
+
+// ---------------------------------------------------------------- tiled path
+constexpr int kBT = 64;           // query rows / keys per block
+constexpr int kBwdThreads = 256;  // 16 x 16 threads
+
+template <int D>
+struct BwdSmem {
+  static constexpr int kDP = D + 4;         // row stride (floats): 16-byte rows, two-way conflicts at most
+  static constexpr int kSP = kBT + 4;
+  float k[kBT][kDP], v[kBT][kDP], q[kBT][kDP], g[kBT][kDP];
+  float a[kBT][kSP];    // a_ij / N_max     [query][key]
+  float ds[kBT][kSP];   // ds_ij            [query][key]
+  float dst[kBT][kSP];  // ds_ij            [key][query]
+  int bk[kBT][kSP];     // time bucket of each pair [query][key]
+  float drt[kMaxBuckets];
+  long long thr[kMaxBuckets];
+  long long tq[kBT], tk[kBT];
+};
+
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+// rows [r0, r0 + 64) of a [rows, H, D] tensor (row stride `stride` elements)
+// into shared memory as fp32; rows at or past `rows` are zero
+template <int D, typename T>
+__device__ __forceinline__ void stage_rows(float (*dst)[D + 4], const T* src, int r0, int rows, int stride,
+                                           int head) {
+  constexpr int kVec = D / 4;
+  for (int x = threadIdx.x; x < kBT * kVec; x += kBwdThreads) {
+    const int r = x / kVec, c = (x % kVec) * 4;
+    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < rows) {
+      const T* p = src + (size_t)(r0 + r) * stride + (size_t)head * D + c;
+      if constexpr (sizeof(T) == 4) {
+        val = *reinterpret_cast<const float4*>(p);
+      } else {
+        const uint2 raw = *reinterpret_cast<const uint2*>(p);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        val = make_float4(lo.x, lo.y, hi.x, hi.y);
+      }
+    }
+    *reinterpret_cast<float4*>(&dst[r][c]) = val;
+  }
+}
+
+// The DE dims of thread dg in the d_k / d_v / d_q products come in chunks of
+// kC = min(DE, 4): chunk c holds dims kC dg + 16 kC c ..  so the 16 threads of
+// a row read one contiguous span of shared memory.
+template <int DE>
+__device__ __forceinline__ int dim_of(int dg, int e) {
+  constexpr int kC = DE < 4 ? DE : 4;
+  return kC * dg + 16 * kC * (e / kC) + e % kC;
+}
+
+template <int DE>
+__device__ __forceinline__ void lds_dims(const float* row, int dg, float (&x)[DE]) {
+  if constexpr (DE >= 4) {
+#pragma unroll
+    for (int c = 0; c < DE / 4; ++c) {
+      const float4 t = lds4(row + 4 * dg + 64 * c);
+      x[4 * c] = t.x;
+      x[4 * c + 1] = t.y;
+      x[4 * c + 2] = t.z;
+      x[4 * c + 3] = t.w;
+    }
+  } else {
+    const float2 t = *reinterpret_cast<const float2*>(row + 2 * dg);
+    x[0] = t.x;
+    x[1] = t.y;
+  }
+}
+
+// global atomics of one row's DE dims (16- or 8-byte vector adds)
+template <int DE>
+__device__ __forceinline__ void red_add_dims(float* row, int dg, const float (&x)[DE]) {
+  if constexpr (DE >= 4) {
+#pragma unroll
+    for (int c = 0; c < DE / 4; ++c)
+      atomicAdd(reinterpret_cast<float4*>(row + 4 * dg + 64 * c),
+                make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]));
+  } else {
+    atomicAdd(reinterpret_cast<float2*>(row + 2 * dg), make_float2(x[0], x[1]));
+  }
+}
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_tiled_kernel(const AttnArgs a, const BucketTable tab, const BwdOut b) {
+  constexpr int DE = D / 16;  // dims per thread in the d_k / d_v / d_q products
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem_raw);
+  if (a.hdr->status != 0) return;
+  const int tid = threadIdx.x;
+  const int u = blockIdx.x / a.H, head = blockIdx.x % a.H;
+  const int kb = blockIdx.y;
+  const int q0 = a.q_offsets[u];
+  const int n = a.q_offsets[u + 1] - q0;
+  const int j0 = kb * kBT;
+  if (j0 >= n) return;
+  const int hist = n - (a.num_cand ? a.num_cand[u] : 0);
+  const T* q = static_cast<const T*>(a.q) + (size_t)q0 * a.qkv_stride;
+  const T* k = static_cast<const T*>(a.k) + (size_t)q0 * a.qkv_stride;
+  const T* v = static_cast<const T*>(a.v) + (size_t)q0 * a.qkv_stride;
+  const float* g = b.d_o + (size_t)q0 * a.H * D;
+  for (int x = tid; x < kMaxBuckets; x += kBwdThreads) {
+    sm.thr[x] = tab.thr[x];
+    sm.drt[x] = 0.f;
+  }
+  stage_rows<D>(sm.k, k, j0, n, a.qkv_stride, head);
+  stage_rows<D>(sm.v, v, j0, n, a.qkv_stride, head);
+  if (tid < kBT) sm.tk[tid] = a.ts[q0 + min(j0 + tid, n - 1)];
+
+  const int ty = tid >> 4, tx = tid & 15;  // S tile: rows ty + 16 r, keys tx + 16 c
+  const int rg = tid >> 4, dg = tid & 15;  // products: keys / queries 4 rg .. 4 rg + 3, dims dim_of(dg, .)
+  float dk[4][DE], dv[4][DE];
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int e = 0; e < DE; ++e) dk[x][e] = dv[x][e] = 0.f;
+  const float inv_n = 1.f / (float)a.n_max;
+  const int nqb = (n + kBT - 1) / kBT;
+  // history keys are seen by every later row (candidates included); a block
+  // of candidate keys only by the candidates themselves
+  const int qb_end = j0 < hist ? nqb : kb + 1;
+  for (int qb = kb; qb < qb_end; ++qb) {
+    const int i0 = qb * kBT;
+    __syncthreads();  // the previous block pair is done with q, g, a, ds, dst and bk
+    stage_rows<D>(sm.q, q, i0, n, a.qkv_stride, head);
+    stage_rows<D, float>(sm.g, g, i0, n, a.H * D, head);
+    if (tid < kBT) sm.tq[tid] = a.ts[q0 + min(i0 + tid, n - 1)];
+    __syncthreads();
+
+    // S = Q K^T and dP = g V^T on 4 x 4 register tiles
+    float s[4][4], dp[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) s[r][c] = dp[r][c] = 0.f;
+#pragma unroll 2
+    for (int e = 0; e < D; e += 4) {
+      float4 qv[4], gv[4], kv[4], vv[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        qv[r] = lds4(&sm.q[ty + 16 * r][e]);
+        gv[r] = lds4(&sm.g[ty + 16 * r][e]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        kv[c] = lds4(&sm.k[tx + 16 * c][e]);
+        vv[c] = lds4(&sm.v[tx + 16 * c][e]);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          s[r][c] = fmaf(qv[r].x, kv[c].x, fmaf(qv[r].y, kv[c].y, fmaf(qv[r].z, kv[c].z, fmaf(qv[r].w, kv[c].w, s[r][c]))));
+          dp[r][c] = fmaf(gv[r].x, vv[c].x, fmaf(gv[r].y, vv[c].y, fmaf(gv[r].z, vv[c].z, fmaf(gv[r].w, vv[c].w, dp[r][c]))));
+        }
+    }
+
+    // a and ds of the block pair, and each pair's time bucket
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int li = ty + 16 * r, lj = tx + 16 * c;
+        const int i = i0 + li, j = j0 + lj;
+        const bool allowed = i < n && j < n && (i < hist ? j <= i : (j < hist || j == i));
+        float av = 0.f, dsv = 0.f;
+        int bkt = 0;
+        if (allowed) {
+          const int p_i = min(i, hist), p_j = min(j, hist);
+          bkt = bucket_of_dt(sm.thr, sm.tq[li] - sm.tk[lj]);
+          const float sv = a.alpha * s[r][c] + a.rab_pos[p_i - p_j + a.n_max - 1] + a.rab_ts[bkt];
+          const float sig = 1.f / (1.f + expf(-sv));
+          av = sv * sig * inv_n;
+          dsv = dp[r][c] * sig * (1.f + sv * (1.f - sig)) * inv_n;
+        }
+        sm.a[li][lj] = av;
+        sm.ds[li][lj] = dsv;
+        sm.dst[lj][li] = dsv;
+        sm.bk[li][lj] = bkt;
+      }
+    __syncthreads();
+    // Bias gradients from the ds tile (ds is 0 outside the allowed set).
+    // d rab_pos: thread w < 127 sums the pairs with p_i - p_j = wbase + w; in
+    // row i that is key position p_i - wbase - w, or the row's own key when
+    // that position is the history length (candidates sit at position h).
+    // d rab_ts: the other 128 threads fold 32 columns of one row each (the
+    // bucket only changes near the diagonal), warp-aggregated when all lanes
+    // share the bucket.
+    if (tid < 127) {
+      const int wbase = min(i0, hist) - min(j0 + kBT - 1, hist);
+      const int w = tid;
+      float acc = 0.f;
+      for (int li = 0; li < kBT; ++li) {
+        const int i = i0 + li;
+        const int pj = min(i, hist) - wbase - w;
+        // a history key at position pj, or (pj == h) a candidate row's own key
+        const bool key = pj >= 0 && (pj < hist || (pj == hist && i >= hist));
+        const int lj = (pj < hist ? pj : i) - j0;
+        if (key && lj >= 0 && lj < kBT) acc += sm.ds[li][lj];
+      }
+      if (acc != 0.f) atomicAdd(b.d_rp + wbase + w + a.n_max - 1, acc);
+    } else if (tid >= 128) {
+      const int t = tid - 128;
+      const int li = t >> 1, c0 = (t & 1) * 32;
+      // lane l starts at column l of its half: the lanes' reads fall in 32 distinct banks
+      const int rot = tid & 31;
+      int run_b = sm.bk[li][c0 + rot];
+      float run_v = 0.f;
+      for (int x = 0; x < 32; ++x) {
+        const int c = c0 + ((x + rot) & 31);
+        const int bb = sm.bk[li][c];
+        if (bb != run_b) {
+          if (run_v != 0.f) atomicAdd(&sm.drt[run_b], run_v);
+          run_b = bb;
+          run_v = 0.f;
+        }
+        run_v += sm.ds[li][c];
+      }
+      // the last run goes through the warp aggregate when every lane shares its bucket
+      const unsigned same = __match_any_sync(~0u, run_b);
+      if (same == ~0u) {
+        float x = run_v;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(~0u, x, o);
+        if ((tid & 31) == 0 && x != 0.f) atomicAdd(&sm.drt[run_b], x);
+      } else if (run_v != 0.f) {
+        atomicAdd(&sm.drt[run_b], run_v);
+      }
+    }
+
+    // d_v += a^T g, d_k += ds^T Q (keys 4 rg .. 4 rg + 3)
+#pragma unroll 4
+    for (int i = 0; i < kBT; ++i) {
+      const float4 av = lds4(&sm.a[i][4 * rg]);
+      const float4 dsv = lds4(&sm.ds[i][4 * rg]);
+      float gr[DE], qr[DE];
+      lds_dims(sm.g[i], dg, gr);
+      lds_dims(sm.q[i], dg, qr);
+      const float aw[4] = {av.x, av.y, av.z, av.w};
+      const float dw[4] = {dsv.x, dsv.y, dsv.z, dsv.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int e = 0; e < DE; ++e) {
+          dv[x][e] = fmaf(aw[x], gr[e], dv[x][e]);
+          dk[x][e] = fmaf(dw[x], qr[e], dk[x][e]);
+        }
+    }
+    // d_q of this query block += alpha ds K (queries 4 rg .. 4 rg + 3)
+    float dq[4][DE];
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int e = 0; e < DE; ++e) dq[x][e] = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < kBT; ++j) {
+      const float4 dsv = lds4(&sm.dst[j][4 * rg]);
+      float kr[DE];
+      lds_dims(sm.k[j], dg, kr);
+      const float dw[4] = {dsv.x, dsv.y, dsv.z, dsv.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int e = 0; e < DE; ++e) dq[x][e] = fmaf(dw[x], kr[e], dq[x][e]);
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int i = i0 + 4 * rg + x;
+      if (i < n) {
+#pragma unroll
+        for (int e = 0; e < DE; ++e) dq[x][e] *= a.alpha;
+        red_add_dims(b.dq + ((size_t)(q0 + i) * a.H + head) * D, dg, dq[x]);
+      }
+    }
+  }
+  // this CTA owns d_k and d_v of its keys
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const int j = j0 + 4 * rg + x;
+    if (j < n) {
+      float* pk = b.dk + ((size_t)(q0 + j) * a.H + head) * D;
+      float* pv = b.dv + ((size_t)(q0 + j) * a.H + head) * D;
+#pragma unroll
+      for (int e = 0; e < DE; ++e) {
+        pk[dim_of<DE>(dg, e)] = a.alpha * dk[x][e];
+        pv[dim_of<DE>(dg, e)] = dv[x][e];
+      }
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < a.nb; x += kBwdThreads)
+    if (sm.drt[x] != 0.f) atomicAdd(b.d_rt + x, sm.drt[x]);
+}
+
 }  // namespace
 
 cudaError_t launch_attn_bwd(const AttnArgs& a, const BucketTable& thr, const float* d_o, float* dq, float* dk,
                             float* dv, float* d_rp, float* d_rt, cudaStream_t s) {
   BwdOut b{d_o, dq, dk, dv, d_rp, d_rt};
+  if ((a.d == 32 || a.d == 64 || a.d == 128) && a.T_q > 0) {
+    if (cudaMemsetAsync(dq, 0, sizeof(float) * (size_t)a.T_q * a.H * a.d, s) != cudaSuccess) return cudaGetLastError();
+    const int max_blocks = (a.n_max + kBT - 1) / kBT;  // key blocks of the longest user
+    const dim3 grid(a.B * a.H, max_blocks);            // block 0 of every user first: the longest CTAs lead
+    auto go = [&](auto kern, size_t smem) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      kern<<<grid, kBwdThreads, smem, s>>>(a, thr, b);
+    };
+    if (a.d == 32) {
+      if (a.in_bf16) go(attn_bwd_tiled_kernel<32, __nv_bfloat16>, sizeof(BwdSmem<32>));
+      else go(attn_bwd_tiled_kernel<32, float>, sizeof(BwdSmem<32>));
+    } else if (a.d == 64) {
+      if (a.in_bf16) go(attn_bwd_tiled_kernel<64, __nv_bfloat16>, sizeof(BwdSmem<64>));
+      else go(attn_bwd_tiled_kernel<64, float>, sizeof(BwdSmem<64>));
+    } else {
+      if (a.in_bf16) go(attn_bwd_tiled_kernel<128, __nv_bfloat16>, sizeof(BwdSmem<128>));
+      else go(attn_bwd_tiled_kernel<128, float>, sizeof(BwdSmem<128>));
+    }
+    return cudaGetLastError();
+  }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

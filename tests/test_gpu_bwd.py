@@ -36,6 +36,9 @@ def run(b, seed):
     ([37, 64], None, 2, 32, torch.float32),
     ([50, 1, 77], [10, 0, 77], 2, 32, torch.float32),
     ([300, 129], [40, 0], 4, 128, torch.bfloat16),
+    ([200, 65, 128], [70, 0, 1], 2, 64, torch.float32),
+    ([64, 130], [64, 3], 1, 128, torch.float32),
+    ([40, 9], [5, 0], 1, 48, torch.float32),       # head dim outside the tiled kernel's set
 ])
 def test_gradients_match_oracle(lengths, cands, H, d, dtype):
     rng = np.random.default_rng(sum(lengths))
