@@ -27,6 +27,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "device_common.cuh"
 #include "hstu_internal.h"
@@ -276,6 +277,45 @@ __device__ __forceinline__ void stage_rows(float (*dst)[D + 4], const T* src, in
   }
 }
 
+// A query block's rows in registers: a thread holds chunks tid + 256 x of
+// 4 elements (fp32 as float4, bf16 as 4 packed halves), so the next block's
+// loads are in flight while the current block's d_q product runs.
+template <int D, typename T>
+struct RowRegs {
+  static constexpr int kN = kBT * (D / 4) / kBwdThreads;
+  using V = typename std::conditional<sizeof(T) == 4, float4, uint2>::type;
+  V v[kN];
+  __device__ __forceinline__ void load(const T* src, int r0, int rows, int stride, int head) {
+#pragma unroll
+    for (int x = 0; x < kN; ++x) {
+      const int id = threadIdx.x + kBwdThreads * x;
+      const int r = id / (D / 4), c = (id % (D / 4)) * 4;
+      if (r0 + r < rows) {
+        v[x] = *reinterpret_cast<const V*>(src + (size_t)(r0 + r) * stride + (size_t)head * D + c);
+      } else {
+        if constexpr (sizeof(T) == 4) v[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+        else v[x] = make_uint2(0u, 0u);
+      }
+    }
+  }
+  __device__ __forceinline__ void store(float (*dst)[D + 4]) const {
+#pragma unroll
+    for (int x = 0; x < kN; ++x) {
+      const int id = threadIdx.x + kBwdThreads * x;
+      const int r = id / (D / 4), c = (id % (D / 4)) * 4;
+      float4 val;
+      if constexpr (sizeof(T) == 4) {
+        val = v[x];
+      } else {
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v[x].x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v[x].y));
+        val = make_float4(lo.x, lo.y, hi.x, hi.y);
+      }
+      *reinterpret_cast<float4*>(&dst[r][c]) = val;
+    }
+  }
+};
+
 // The DE dims of thread dg in the d_k / d_v / d_q products come in chunks of
 // kC = min(DE, 4): chunk c holds dims kC dg + 16 kC c ..  so the 16 threads of
 // a row read one contiguous span of shared memory.
@@ -355,12 +395,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // history keys are seen by every later row (candidates included); a block
   // of candidate keys only by the candidates themselves
   const int qb_end = j0 < hist ? nqb : kb + 1;
+  RowRegs<D, T> nq;
+  RowRegs<D, float> ng;
+  long long nts = 0;
+  auto fetch = [&](int qb) {
+    nq.load(q, qb * kBT, n, a.qkv_stride, head);
+    ng.load(g, qb * kBT, n, a.H * D, head);
+    if (tid < kBT) nts = a.ts[q0 + min(qb * kBT + tid, n - 1)];
+  };
+  fetch(kb);
   for (int qb = kb; qb < qb_end; ++qb) {
     const int i0 = qb * kBT;
     __syncthreads();  // the previous block pair is done with q, g, a, ds, dst and bk
-    stage_rows<D>(sm.q, q, i0, n, a.qkv_stride, head);
-    stage_rows<D, float>(sm.g, g, i0, n, a.H * D, head);
-    if (tid < kBT) sm.tq[tid] = a.ts[q0 + min(i0 + tid, n - 1)];
+    nq.store(sm.q);
+    ng.store(sm.g);
+    if (tid < kBT) sm.tq[tid] = nts;
     __syncthreads();
 
     // S = Q K^T and dP = g V^T on 4 x 4 register tiles
@@ -482,6 +531,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dk[x][e] = fmaf(dw[x], qr[e], dk[x][e]);
         }
     }
+    // the next query block's rows load while d_q is formed
+    if (qb + 1 < qb_end) fetch(qb + 1);
     // d_q of this query block += alpha ds K (queries 4 rg .. 4 rg + 3)
     float dq[4][DE];
 #pragma unroll
