@@ -22,16 +22,19 @@
 // the candidate's own term a_ii v_i is added by the epilogue, so no tile of
 // the candidate x candidate block is ever issued.
 //
-// Warp roles (576 threads): warps 0-15 elementwise in four warpgroups, one
+// Warp roles (608 threads): warps 0-15 elementwise in four warpgroups, one
 // per (query tile, 64-key half of every key tile) (thread = query row = TMEM
 // lane; a warp reaches the lanes of its rank in the warpgroup), warp 16
-// producer (Q once; K/V
-// through a 2-stage ring by TMA, the paged prefix page by page; per key tile
-// it also stages the keys' timestamps and a window of 0.5*rab_pos in shared
-// memory), warp 17 MMA issuer and TMEM owner.  Tensor memory holds S_A, S_B,
-// O_A, O_B (4 x 128 columns); while one warpgroup turns S into P the tensor
-// core runs the other tile's GEMMs, and each 64-key half of P goes to the
-// A.V GEMM as soon as it is written.  Every wait is bounded (about 2 s), after
+// producer (Q once; K/V through a 2-stage ring by TMA, the paged prefix page
+// by page; per key tile it also stages the keys' timestamps and a window of
+// 0.5*rab_pos in shared memory), warps 17 and 18 the MMA issuers of query
+// tiles A and B (warp 17 owns tensor memory).  Tensor memory holds S_A, S_B,
+// O_A, O_B (4 x 128 columns).  Each tile's issuer follows its own two
+// warpgroups: as soon as one 64-key half of P is written it issues that
+// half's A.V GEMM and then the next key tile's S for the same 64 columns
+// (N = 64), so a warpgroup waits only for its own half, and neither tile's
+// GEMMs queue behind the other tile's waits.  A K/V stage is released once
+// both tiles' GEMMs that read it completed.  Every wait is bounded (about 2 s), after
 // which the kernel reports HSTU_ERR_TIMEOUT and winds down.
 //
 // Elementwise work per score: hb = s/2 = (alpha/2) S + 0.5 (rab_pos + rab_ts)
@@ -61,9 +64,10 @@ namespace {
 
 constexpr int kQTiles = 2;
 constexpr int kEwWarps = 16;                 // 4 warpgroups: (query tile, 64-column half)
-constexpr int kThreads = 32 * (kEwWarps + 2);
+constexpr int kThreads = 32 * (kEwWarps + 3);
 constexpr int kProducerWarp = kEwWarps;
-constexpr int kMmaWarp = kEwWarps + 1;
+constexpr int kMmaWarp = kEwWarps + 1;   // MMA issuer of tile A, TMEM owner
+constexpr int kMmaWarpB = kEwWarps + 2;  // MMA issuer of tile B
 constexpr int kStages = 2;
 constexpr int kTileBytes = kTile * 128 * 2;  // 128 rows x 128 bf16 = 32 KB
 constexpr int kHalfBytes = kTile * 128;      // 128 rows x 64 bf16: one 128B-swizzled box
@@ -89,11 +93,11 @@ struct __align__(1024) Smem {
   uint64_t bar_k_full[kStages];
   uint64_t bar_v_full[kStages];
   uint64_t bar_meta_full[kStages];
-  uint64_t bar_kv_empty[kStages];
-  uint64_t bar_s_full[kQTiles];
+  uint64_t bar_kv_empty[kQTiles][kStages];  // stage released by tile X's GEMMs
+  uint64_t bar_s_full[kQTiles][2];  // S of keys 0-63 / 64-127 written
   uint64_t bar_p_lo[kQTiles];  // P of keys 0-63 written
   uint64_t bar_p_hi[kQTiles];  // P of keys 64-127 written
-  uint64_t bar_o_full;
+  uint64_t bar_o_full[kQTiles];
   uint32_t tmem_base;
   int abort;
 };
@@ -294,14 +298,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.bar_k_full[s], 1);
       mbar_init(&sm.bar_v_full[s], 1);
       mbar_init(&sm.bar_meta_full[s], 32);
-      mbar_init(&sm.bar_kv_empty[s], 1);
+      mbar_init(&sm.bar_kv_empty[0][s], 1);
+      mbar_init(&sm.bar_kv_empty[1][s], 1);
     }
     for (int x = 0; x < kQTiles; ++x) {
-      mbar_init(&sm.bar_s_full[x], 1);
+      mbar_init(&sm.bar_s_full[x][0], 1);
+      mbar_init(&sm.bar_s_full[x][1], 1);
       mbar_init(&sm.bar_p_lo[x], kTile);
       mbar_init(&sm.bar_p_hi[x], kTile);
     }
-    mbar_init(&sm.bar_o_full, 1);
+    mbar_init(&sm.bar_o_full[0], 1);
+    mbar_init(&sm.bar_o_full[1], 1);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -372,7 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int k0, width;
       key_tile(gA, tb + t, k0, width);
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(&sm.bar_kv_empty[s], ph ^ 1, abort_flag, a.hdr, 1);
+      // the stage's previous tile (t - kStages) is released by each query tile that used it
+      if (lane == 0 && t - kStages < cA) ok = mbar_wait(&sm.bar_kv_empty[0][s], ph ^ 1, abort_flag, a.hdr, 1);
+      if (lane == 0 && ok && t - kStages < cB) ok = mbar_wait(&sm.bar_kv_empty[1][s], ph ^ 1, abort_flag, a.hdr, 1);
       ok = __shfl_sync(~0u, ok, 0);
       if (!ok) break;
       uint8_t* kd = sm.k[s];
@@ -461,67 +470,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp || warp == kMmaWarpB) {
+    // ------------------------------------------------------------------ MMA issuers, one per query tile
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
+      const int x = warp == kMmaWarp ? 0 : 1;
+      const int c = x == 0 ? cA : cB;
       constexpr uint32_t idesc_pv = idesc_bf16(128, 128, 0, 1);
-      const int cnt[kQTiles] = {cA, cB};
-      auto issue_s = [&](int x, int t) {
+      constexpr uint32_t idesc_qk_half = idesc_bf16(128, 64, 0, 0);
+      // S_X over keys [64 h, 64 h + 64) of tile t into columns 64 h .. 64 h + 63:
+      // issued per half so that each half follows its own half of P into the
+      // A.V GEMM (the half's columns hold that P until then)
+      auto issue_s_half = [&](int t, int h) {
         const uint32_t q_base = smem_u32(sm.q[x]);
-        const uint32_t k_base = smem_u32(sm.k[t % kStages]);
+        const uint32_t k_base = smem_u32(sm.k[t % kStages]) + h * 64 * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(tmem + x * 128, sw128_desc(q_base + off, 16, 1024), sw128_desc(k_base + off, 16, 1024),
-                 idesc_qk, kk > 0);
+          mma_ss(tmem + x * 128 + 64 * h, sw128_desc(q_base + off, 16, 1024), sw128_desc(k_base + off, 16, 1024),
+                 idesc_qk_half, kk > 0);
         }
-        mma_commit(&sm.bar_s_full[x]);
+        mma_commit(&sm.bar_s_full[x][h]);
       };
       // O_X += P_X V over keys [64 h, 64 h + 64): P at columns 64 h .. 64 h + 31 of
       // S_X (16 keys per 8 columns), V rows 64 h..
-      auto issue_pv_half = [&](int x, int t, int h) {
+      auto issue_pv_half = [&](int t, int h) {
         const uint32_t v_base = smem_u32(sm.v[t % kStages]);
 #pragma unroll
         for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
           mma_ts(tmem + 256 + x * 128, tmem + x * 128 + 64 * h + (kk - 4 * h) * 8,
                  sw128_desc(v_base + kk * 2048, kHalfBytes, 1024), idesc_pv, (t > 0 || kk > 0));
       };
-      bool ok = cT == 0 || mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 2);
-      if (ok && cT > 0) ok = mbar_wait(&sm.bar_k_full[0], 0, abort_flag, a.hdr, 3);
+      bool ok = c == 0 || mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 2);
+      if (ok && c > 0) ok = mbar_wait(&sm.bar_k_full[0], 0, abort_flag, a.hdr, 3);
       tc_fence_after();
-      if (ok && cT > 0) {
-        for (int x = 0; x < kQTiles; ++x)
-          if (cnt[x] > 0) issue_s(x, 0);
+      if (ok && c > 0) {
+        issue_s_half(0, 0);
+        issue_s_half(0, 1);
       }
-      for (int t = 0; ok && t < cT; ++t) {
+      for (int t = 0; ok && t < c; ++t) {
         const int s = t % kStages;
-        bool v_ready = false, k_next_ready = false;
-        for (int x = 0; ok && x < kQTiles; ++x) {
-          if (t >= cnt[x]) continue;
-          ok = mbar_wait(&sm.bar_p_lo[x], t & 1, abort_flag, a.hdr, 4);
-          if (ok && !v_ready) ok = v_ready = mbar_wait(&sm.bar_v_full[s], (t / kStages) & 1, abort_flag, a.hdr, 5);
+        ok = mbar_wait(&sm.bar_p_lo[x], t & 1, abort_flag, a.hdr, 4);
+        if (ok) ok = mbar_wait(&sm.bar_v_full[s], (t / kStages) & 1, abort_flag, a.hdr, 5);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv_half(t, 0);
+        const bool next = t + 1 < c;
+        if (next) {
+          ok = mbar_wait(&sm.bar_k_full[(t + 1) % kStages], ((t + 1) / kStages) & 1, abort_flag, a.hdr, 3);
           if (!ok) break;
           tc_fence_after();
-          issue_pv_half(x, t, 0);
-          ok = mbar_wait(&sm.bar_p_hi[x], t & 1, abort_flag, a.hdr, 4);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv_half(x, t, 1);
-          if (t + 1 < cnt[x]) {
-            if (!k_next_ready)
-              ok = k_next_ready = mbar_wait(&sm.bar_k_full[(t + 1) % kStages], ((t + 1) / kStages) & 1,
-                                            abort_flag, a.hdr, 3);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(x, t + 1);
-          }
+          issue_s_half(t + 1, 0);
         }
-        if (ok) mma_commit(&sm.bar_kv_empty[s]);
+        ok = mbar_wait(&sm.bar_p_hi[x], t & 1, abort_flag, a.hdr, 4);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv_half(t, 1);
+        if (next) issue_s_half(t + 1, 1);
+        mma_commit(&sm.bar_kv_empty[x][s]);
       }
-      mma_commit(&sm.bar_o_full);
+      mma_commit(&sm.bar_o_full[x]);
       // tensor memory is freed below only after every issued MMA completed
-      mbar_wait(&sm.bar_o_full, 0, nullptr, a.hdr, 8);
+      mbar_wait(&sm.bar_o_full[x], 0, nullptr, a.hdr, 8);
     }
     __syncwarp();
   } else {
@@ -554,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int k0, width;
       key_tile(g, tb + t, k0, width);
       ok = mbar_wait(&sm.bar_meta_full[s], (t / kStages) & 1, abort_flag, a.hdr, 6);
-      ok = ok && mbar_wait(&sm.bar_s_full[x], t & 1, abort_flag, a.hdr, 6);
+      ok = ok && mbar_wait(&sm.bar_s_full[x][half], t & 1, abort_flag, a.hdr, 6);
       ok = ew_all(ok, group);
       if (!ok) break;
       tc_fence_after();
@@ -619,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(half == 0 ? &sm.bar_p_lo[x] : &sm.bar_p_hi[x]);
     }
     if (ok && cT > 0) {
-      ok = ew_all(mbar_wait(&sm.bar_o_full, 0, abort_flag, a.hdr, 7), group);
+      ok = ew_all(mbar_wait(&sm.bar_o_full[x], 0, abort_flag, a.hdr, 7), group);
       tc_fence_after();
     }
     if (ok && exists) {
