@@ -399,25 +399,47 @@ def run_paged_bench(args, device):
         for x in dl:
             call(x, 0)
     torch.cuda.synchronize()
-    ev = []
+    # whole layers as a caller runs them (three Python calls per layer: plan, attention, epilogue)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(steps):
         for x in dl:
-            call(x, _lib.F_STAGE_PLAN)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            call(x, _lib.F_STAGE_ATTN)
-            b.record(stream)
-            call(x, _lib.F_STAGE_EPILOGUE)
-            ev.append((a, b))
+            call(x, 0)
     t1.record(stream)
     torch.cuda.synchronize()
     status = hstu.hstu_check_device_error(ws)
     if status != 0:
         raise RuntimeError(f"paged device status {status}")
     ms_layer = t0.elapsed_time(t1) / (steps * len(dl))
-    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    # The attention kernel alone: its launches for the 8 layers captured in a CUDA
+    # graph and replayed, so no host time (argument marshalling, tensor-map
+    # encoding) falls between the events.  Every layer has the same users and
+    # cached lengths, so one plan serves all of them.
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        call(dl[0], _lib.F_STAGE_PLAN)
+        for x in dl:
+            call(x, _lib.F_STAGE_ATTN)
+        cap.synchronize()
+        with torch.cuda.graph(graph, stream=cap):
+            for x in dl:
+                call(x, _lib.F_STAGE_ATTN)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    attn_ms = a.elapsed_time(b) / (steps * len(dl))
+    status = hstu.hstu_check_device_error(ws)
+    if status != 0:
+        raise RuntimeError(f"paged device status {status}")
+    del graph
     kv_bytes = int(sum(2 * int(c) * 4 * 128 * 2 for c in pb0.cached_lens))
     new_bytes = T * 512 * 2 * 4 + int(pb0.ts_offsets[-1]) * 8
     alg_bytes = kv_bytes + new_bytes
@@ -431,7 +453,9 @@ def run_paged_bench(args, device):
                          "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                          "frac": round(achieved / float(peaks["hbm_gbs"]), 4),
                          "peak_source": f"{kind} hbm_gbs", "bytes_per_launch": alg_bytes,
-                         "launch_ms": round(attn_ms, 4), "traffic": PAGED_TRAFFIC_BYTES}}
+                         "launch_ms": round(attn_ms, 4), "timing": "CUDA-graph replay of the 8 layers' "
+                                                                       "attention launches",
+                         "traffic": PAGED_TRAFFIC_BYTES}}
 
 
 def run_glue_bench(args, device):
