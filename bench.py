@@ -41,8 +41,8 @@ TILE = 128
 # captures summarised in profiles/attn_sm100_stack8.md and
 # profiles/attn_sm100_paged.md; set to None when the kernel changes until it
 # is captured again.
-ATTN_TRAFFIC_BYTES = 404_022_272 + 83_838_464
-PAGED_TRAFFIC_BYTES = 114_777_088 + 6_897_920
+ATTN_TRAFFIC_BYTES = 392_002_560 + 71_595_776
+PAGED_TRAFFIC_BYTES = 114_754_560 + 5_426_432
 
 
 def allowed_pairs(lengths, cands=None):
