@@ -289,29 +289,55 @@ def run_ours(args, rank, world, device):
         h_off = torch.from_numpy(b0.seq_offsets.astype(np.int32)).pin_memory()
         h_ts = torch.from_numpy(b0.timestamps).pin_memory()
         h_out = [torch.empty(T, H * d, dtype=b0.q.dtype).pin_memory() for _ in range(L)]
-        d_in = {k: torch.empty_like(v, device=device) for k, v in host[0].items()}
+        # two device input sets and two output buffers: layer l + 1's inputs copy
+        # in on one stream while layer l computes, and each output copies out on a
+        # third stream (host-to-device and device-to-host run at once)
+        d_in = [{k: torch.empty_like(v, device=device) for k, v in host[0].items()} for _ in range(2)]
         d_off = torch.empty_like(h_off, device=device)
         d_ts = torch.empty_like(h_ts, device=device)
-        d_out = torch.empty(T, H * d, dtype=b0.q.dtype, device=device)
+        d_out = [torch.empty(T, H * d, dtype=b0.q.dtype, device=device) for _ in range(2)]
+        s_h2d, s_d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer set j landed
+        ev_used = [torch.cuda.Event() for _ in range(2)]   # compute done with buffer set j
+        ev_out = [torch.cuda.Event() for _ in range(2)]    # output buffer j copied out
+        for j in range(2):
+            ev_used[j].record(stream)
+            ev_out[j].record(stream)
         h2d = d2h = 0
 
         def e2e_step(count):
             nonlocal h2d, d2h
-            d_off.copy_(h_off, non_blocking=True)
-            d_ts.copy_(h_ts, non_blocking=True)
+            with torch.cuda.stream(s_h2d):
+                s_h2d.wait_stream(stream)
+                d_off.copy_(h_off, non_blocking=True)
+                d_ts.copy_(h_ts, non_blocking=True)
             if count:
                 h2d += h_off.numel() * 4 + h_ts.numel() * 8
             for l in range(L):
-                for k_, v_ in host[l].items():
-                    d_in[k_].copy_(v_, non_blocking=True)
-                    if count:
-                        h2d += v_.numel() * v_.element_size()
-                hstu.hstu_attn_fwd(d_in["q"], d_in["k"], d_in["v"], d_in["u"], d_off, d_ts, d_in["rab_pos"],
-                                   d_in["rab_ts"], n_max=b0.n_max, alpha=b0.alpha, max_seq_len=b0.max_seq_len,
-                                   out=d_out, workspace=ws)
-                h_out[l].copy_(d_out, non_blocking=True)
+                j = l % 2
+                with torch.cuda.stream(s_h2d):
+                    s_h2d.wait_event(ev_used[j])
+                    for k_, v_ in host[l].items():
+                        d_in[j][k_].copy_(v_, non_blocking=True)
+                        if count:
+                            h2d += v_.numel() * v_.element_size()
+                    ev_in[j].record(s_h2d)
+                stream.wait_event(ev_in[j])
+                stream.wait_event(ev_out[j])
+                x = d_in[j]
+                hstu.hstu_attn_fwd(x["q"], x["k"], x["v"], x["u"], d_off, d_ts, x["rab_pos"], x["rab_ts"],
+                                   n_max=b0.n_max, alpha=b0.alpha, max_seq_len=b0.max_seq_len, out=d_out[j],
+                                   workspace=ws)
+                ev_used[j].record(stream)
+                with torch.cuda.stream(s_d2h):
+                    s_d2h.wait_event(ev_used[j])
+                    h_out[l].copy_(d_out[j], non_blocking=True)
+                    ev_out[j].record(s_d2h)
                 if count:
-                    d2h += d_out.numel() * d_out.element_size()
+                    d2h += d_out[j].numel() * d_out[j].element_size()
+            # the step ends when its last output is on the host
+            stream.wait_stream(s_d2h)
+            stream.wait_stream(s_h2d)
 
         e2e_step(False)
         torch.cuda.synchronize()
