@@ -53,7 +53,10 @@ __device__ __forceinline__ int check_user(const AttnArgs& a, int u, int& n, int&
 }
 
 // work list: per user, blocks of kItemRows query rows, each expanded to
-// H heads x num_splits splits; counting sort by cost (key tiles per split)
+// H heads x num_splits splits; counting sort by cost (key tiles per split).
+// The block's threads form min(B, 256) groups; group g takes users g, g + G, ..
+// and its threads share each user's query blocks, so a batch of a few long
+// users is spread over the whole block as well as a batch of many short ones.
 __device__ void build_schedule(const AttnArgs& a, int* hist, int* start) {
   const int tid = threadIdx.x;
   for (int x = tid; x < kCostBins; x += blockDim.x) hist[x] = 0;
@@ -78,40 +81,57 @@ __device__ void build_schedule(const AttnArgs& a, int* hist, int* start) {
       c = max(c, key_tiles_of(g.L, g.n, g.h, m * tiles_per_item + x));
     return min(ceil_div(c, a.num_splits), kCostBins - 1);
   };
-  for (int u = tid; u < a.B; u += blockDim.x) {
-    const UserGeom g = user_geom(u);
-    for (int m = ceil_div(g.nq, kItemRows) - 1; m >= 0; --m) atomicAdd(&hist[cost_of(g, m)], per);
-  }
+  const int groups = min(a.B, (int)blockDim.x);
+  const int group_size = blockDim.x / groups;
+  const int grp = tid / group_size, sub = tid % group_size;
+  const bool active = grp < groups;
+  if (active)
+    for (int u = grp; u < a.B; u += groups) {
+      const UserGeom g = user_geom(u);
+      for (int m = sub; m < ceil_div(g.nq, kItemRows); m += group_size) atomicAdd(&hist[cost_of(g, m)], per);
+    }
   __syncthreads();
-  // start[c] = number of items with a cost above c (descending order)
-  if (tid < 32) {
-    int carry = 0;
-    for (int base = kCostBins - 32; base >= 0; base -= 32) {
-      const int c = base + 31 - tid;  // lane 0 takes the highest cost of the chunk
-      const int v = hist[c];
-      int incl = v;
+  // start[c] = number of items with a cost above c (descending order): thread t
+  // owns the 4 bins 1023 - 4t .. 1020 - 4t; warp scans, then the 8 warp totals
+  static_assert(kCostBins == 4 * kPlanThreads, "four cost bins per thread");
+  __shared__ int warp_sum[kPlanThreads / 32];
+  const int lane = tid & 31, wid = tid >> 5;
+  int v[4], local = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(~0u, incl, o);
-        if (tid >= o) incl += y;
-      }
-      start[c] = carry + incl - v;
-      carry += __shfl_sync(~0u, incl, 31);
-    }
-    if (tid == 0) a.hdr->n_items = min(carry, a.max_items);
+  for (int k = 0; k < 4; ++k) {
+    v[k] = hist[kCostBins - 1 - (4 * tid + k)];
+    local += v[k];
   }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(~0u, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sum[wid] = incl;
   __syncthreads();
-  for (int u = tid; u < a.B; u += blockDim.x) {
-    const UserGeom g = user_geom(u);
-    for (int m = ceil_div(g.nq, kItemRows) - 1; m >= 0; --m) {
-      const int pos = atomicAdd(&start[cost_of(g, m)], per);
-      for (int h = 0; h < a.H; ++h)
-        for (int s = 0; s < a.num_splits; ++s) {
-          const int idx = pos + h * a.num_splits + s;
-          if (idx < a.max_items) a.items[idx] = WorkItem{u, m, h, s};
-        }
-    }
+  int before = 0;
+  for (int w = 0; w < wid; ++w) before += warp_sum[w];
+  int run = before + incl - local;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    start[kCostBins - 1 - (4 * tid + k)] = run;
+    run += v[k];
   }
+  if (tid == blockDim.x - 1) a.hdr->n_items = min(run, a.max_items);
+  __syncthreads();
+  if (active)
+    for (int u = grp; u < a.B; u += groups) {
+      const UserGeom g = user_geom(u);
+      for (int m = sub; m < ceil_div(g.nq, kItemRows); m += group_size) {
+        const int pos = atomicAdd(&start[cost_of(g, m)], per);
+        for (int h = 0; h < a.H; ++h)
+          for (int s = 0; s < a.num_splits; ++s) {
+            const int idx = pos + h * a.num_splits + s;
+            if (idx < a.max_items) a.items[idx] = WorkItem{u, m, h, s};
+          }
+      }
+    }
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const AttnArgs a, int parts, int schedule) {
