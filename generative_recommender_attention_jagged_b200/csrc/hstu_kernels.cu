@@ -406,13 +406,29 @@ __global__ void __launch_bounds__(256) epilogue_vec_kernel(const AttnArgs a) {
   const size_t split_stride = (size_t)a.T_q * D;
   for (int row = blockIdx.x * warps_per_block + (threadIdx.x >> 5); row < a.T_q;
        row += gridDim.x * warps_per_block) {
+    // the row's gate u is loaded with its partials, so both latencies overlap;
+    // partials, u and y are touched once (streaming loads and stores)
+    float uv[VPT][4] = {};
+#pragma unroll
+    for (int k = 0; k < VPT && !a.out_raw; ++k) {
+      const TIn* up = static_cast<const TIn*>(a.u) + (size_t)row * a.u_stride + 128 * k + 4 * lane;
+      if constexpr (sizeof(TIn) == 2) {
+        const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(up));
+        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+        uv[k][0] = __low2float(lo); uv[k][1] = __high2float(lo); uv[k][2] = __low2float(hi); uv[k][3] = __high2float(hi);
+      } else {
+        const float4 f = __ldcs(reinterpret_cast<const float4*>(up));
+        uv[k][0] = f.x; uv[k][1] = f.y; uv[k][2] = f.z; uv[k][3] = f.w;
+      }
+    }
     float o[VPT][4];
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const float4* src = reinterpret_cast<const float4*>(a.o_ws + (size_t)row * D + 128 * k + 4 * lane);
-      float4 acc = src[0];
+      float4 acc = __ldcs(src);
       for (int sp = 1; sp < a.num_splits; ++sp) {
-        const float4 v = src[sp * split_stride / 4];
+        const float4 v = __ldcs(src + sp * split_stride / 4);
         acc.x += v.x;
         acc.y += v.y;
         acc.z += v.z;
@@ -491,19 +507,9 @@ __global__ void __launch_bounds__(256) epilogue_vec_kernel(const AttnArgs a) {
         const float4 bb = *reinterpret_cast<const float4*>(a.ln_beta + e0);
         b[0] = bb.x; b[1] = bb.y; b[2] = bb.z; b[3] = bb.w;
       }
-      float uv[4], y[4];
-      const TIn* up = static_cast<const TIn*>(a.u) + (size_t)row * a.u_stride + e0;
-      if constexpr (sizeof(TIn) == 2) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(up);
-        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-        uv[0] = __low2float(lo); uv[1] = __high2float(lo); uv[2] = __low2float(hi); uv[3] = __high2float(hi);
-      } else {
-        const float4 f = *reinterpret_cast<const float4*>(up);
-        uv[0] = f.x; uv[1] = f.y; uv[2] = f.z; uv[3] = f.w;
-      }
+      float y[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) y[c] = ((o[k][c] - mean) * rstd * g[c] + b[c]) * uv[c];
+      for (int c = 0; c < 4; ++c) y[c] = ((o[k][c] - mean) * rstd * g[c] + b[c]) * uv[k][c];
       TOut* out = static_cast<TOut*>(a.out) + (size_t)row * D + e0;
       if constexpr (sizeof(TOut) == 2) {
         __nv_bfloat162 lo = __floats2bfloat162_rn(y[0], y[1]);
@@ -511,9 +517,9 @@ __global__ void __launch_bounds__(256) epilogue_vec_kernel(const AttnArgs a) {
         uint2 raw;
         raw.x = *reinterpret_cast<uint32_t*>(&lo);
         raw.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(out) = raw;
+        __stcs(reinterpret_cast<uint2*>(out), raw);
       } else {
-        *reinterpret_cast<float4*>(out) = make_float4(y[0], y[1], y[2], y[3]);
+        __stcs(reinterpret_cast<float4*>(out), make_float4(y[0], y[1], y[2], y[3]));
       }
     }
   }
