@@ -396,6 +396,18 @@ __global__ void __launch_bounds__(256) epilogue_kernel(const AttnArgs a) {
 // Vectorised epilogue for D = H*d a multiple of 128 (D = 128 * VPT): lane l
 // holds features 128 k + 4 l .. 128 k + 4 l + 3 (float4 loads of the partial
 // sums, 8-byte loads/stores of bf16).  Same arithmetic as epilogue_kernel.
+// 4 consecutive features as fp32 (one 8-byte load for bf16, 16-byte for fp32)
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float (&x)[4]) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(p);
+  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+  x[0] = lo.x; x[1] = lo.y; x[2] = hi.x; x[3] = hi.y;
+}
+__device__ __forceinline__ void load4(const float* p, float (&x)[4]) {
+  const float4 f = *reinterpret_cast<const float4*>(p);
+  x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+}
+
 template <int VPT, typename TIn, typename TOut>
 __global__ void __launch_bounds__(256) epilogue_vec_kernel(const AttnArgs a) {
   if (a.hdr->status != 0) return;
@@ -444,29 +456,35 @@ __global__ void __launch_bounds__(256) epilogue_vec_kernel(const AttnArgs a) {
       const int q0 = a.q_offsets[u];
       const int nq = a.q_offsets[u + 1] - q0;
       if (row - q0 >= nq - a.num_cand[u]) {
+        // the candidate's own term a_ii v_i per head (position and time
+        // differences are 0): q, k, v of the row in one vector load per chunk;
+        // a lane's 4 features of chunk k belong to head (128 k + 4 lane) / d
         const float bias = a.rab_pos[a.n_max - 1] + a.rab_ts[0];
         const TIn* q = static_cast<const TIn*>(a.q) + (size_t)row * a.qkv_stride;
         const TIn* kk = static_cast<const TIn*>(a.k) + (size_t)row * a.qkv_stride;
         const TIn* v = static_cast<const TIn*>(a.v) + (size_t)row * a.qkv_stride;
-        // head h covers features [h d, (h+1) d); d is a multiple of 4 here
+        float qv[VPT][4], kv[VPT][4], vv[VPT][4];
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+          const int e0 = 128 * k + 4 * lane;
+          load4(q + e0, qv[k]);
+          load4(kk + e0, kv[k]);
+          load4(v + e0, vv[k]);
+        }
         for (int h = 0; h < a.H; ++h) {
           float part = 0.f;
 #pragma unroll
           for (int k = 0; k < VPT; ++k)
+            if ((128 * k + 4 * lane) / a.d == h)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int e = 128 * k + 4 * lane + c;
-              if (e / a.d == h) part = fmaf(to_f(q[e]), to_f(kk[e]), part);
-            }
+              for (int c = 0; c < 4; ++c) part = fmaf(qv[k][c], kv[k][c], part);
           const float sc = a.alpha * warp_sum(part) + bias;
           const float wgt = sc / (1.f + expf(-sc));
 #pragma unroll
           for (int k = 0; k < VPT; ++k)
+            if ((128 * k + 4 * lane) / a.d == h)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int e = 128 * k + 4 * lane + c;
-              if (e / a.d == h) o[k][c] = fmaf(wgt, to_f(v[e]), o[k][c]);
-            }
+              for (int c = 0; c < 4; ++c) o[k][c] = fmaf(wgt, vv[k][c], o[k][c]);
         }
       }
     }
