@@ -119,6 +119,26 @@ def test_bf16_tensor_core_small(lengths, cands):
     assert rel_err(y, want_y) <= BF16_TOL
 
 
+@pytest.mark.parametrize("num_users", [3, 300])
+def test_work_list_for_few_and_many_users(num_users):
+    """The planner's last block builds the work list with its 256 threads in
+    min(B, 256) groups: 3 users leave threads idle (256 = 3 x 85 + 1), 300
+    users give one thread per group and several users per thread.  Every
+    row must come out, with the lengths spanning one to several query blocks."""
+    rng = np.random.default_rng(num_users)
+    if num_users == 3:
+        lengths, cands = [600, 1, 257], [0, 0, 57]
+    else:
+        lengths = rng.integers(1, 300, size=num_users)
+        lengths[::37] = 520                    # a few users with two query blocks
+        cands = np.where(np.arange(num_users) % 5 == 0, np.minimum(lengths, 9), 0)
+    b = small_batch(list(lengths), cands=list(cands), n_max=640, seed=num_users)
+    want_y, want_o = oracle.batch_attn(b, want_o=True)
+    o = host64(run_jagged(b, raw_av=True))
+    assert rel_err(o, want_o) <= BF16_TOL
+    assert np.abs(o.reshape(o.shape[0], -1)).sum(axis=1).min() > 0   # no row left out of the work list
+
+
 def test_bf16_tensor_core_matches_cuda_core_kernel():
     b = small_batch([400, 131, 77], cands=[50, 0, 3], n_max=512, seed=5)
     o_tc = host64(run_jagged(b, raw_av=True))
