@@ -34,7 +34,9 @@
 // half's A.V GEMM and then the next key tile's S for the same 64 columns
 // (N = 64), so a warpgroup waits only for its own half, and neither tile's
 // GEMMs queue behind the other tile's waits.  A K/V stage is released once
-// both tiles' GEMMs that read it completed.  Every wait is bounded (about 2 s), after
+// both tiles' GEMMs that read it completed.  At the end each warpgroup stages
+// its O columns in its tile's (then idle) Q buffer and writes whole 128-byte
+// row segments of the fp32 partial.  Every wait is bounded (about 2 s), after
 // which the kernel reports HSTU_ERR_TIMEOUT and winds down.
 //
 // Elementwise work per score: hb = s/2 = (alpha/2) S + 0.5 (rab_pos + rab_ts)
@@ -124,6 +126,18 @@ __device__ __forceinline__ float4 lds_f4(const float* p) {
                : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
                : "r"(smem_u32(p)));
   return r;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr)
+               : "memory");
+  return r;
+}
+
+// the threads of one elementwise warpgroup wait for each other (barrier 1 + group)
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // the 128 threads of one elementwise warpgroup (0..3) agree on a flag
@@ -543,7 +557,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cnt = x == 0 ? cA : cB;
     const bool exists = x == 0 || hasB;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const bool valid = exists && r < g.nq_rows;
     const int i = min(g.qs + r, g.n - 1);  // rows past the user repeat its last row (discarded)
     const int jmax = i < g.h ? i : g.h - 1;
     const int pr = min(i, g.h);
@@ -631,8 +644,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ew_all(mbar_wait(&sm.bar_o_full[x], 0, abort_flag, a.hdr, 7), group);
       tc_fence_after();
     }
+    // with no key tile nothing waited for Q; it lands in the staging area below
+    if (ok && cT == 0) ok = ew_all(mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 7), group);
     if (ok && exists) {
-      float* orow = a.o_ws + (((size_t)it.split * a.T_q + (g.qrow0 + r)) * a.H + it.head) * kHeadDim;
+      // O of this warpgroup's 64 columns goes out through shared memory, 32
+      // columns at a time: its half of the tile's Q buffer (free once the
+      // tile's GEMMs completed) holds 128 rows x 128 bytes, 16-byte chunk c of
+      // row r at c ^ (r & 7), and each warp then writes whole 128-byte row
+      // segments (a thread's own row would be 32 scattered 16-byte pieces)
+      const uint32_t stage = smem_u32(sm.q[x]) + half * (kTileBytes / 2);
+      const int wq = warp & 3;  // warp rank in the warpgroup
 #pragma unroll 1
       for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
         uint32_t orr[32];
@@ -643,13 +664,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) orr[e] = 0u;
         }
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(orow + ch * 32);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(orr[4 * e]), __uint_as_float(orr[4 * e + 1]),
-                                 __uint_as_float(orr[4 * e + 2]), __uint_as_float(orr[4 * e + 3]));
+        for (int c = 0; c < 8; ++c)
+          sts_v4(stage + r * 128 + ((c ^ (r & 7)) << 4),
+                 make_uint4(orr[4 * c], orr[4 * c + 1], orr[4 * c + 2], orr[4 * c + 3]));
+        named_bar_sync(1 + group, kTile);
+        // lanes 8 i .. 8 i + 7 of a warp write row rr's 8 chunks
+#pragma unroll 1
+        for (int rr = 4 * wq + (lane >> 3); rr < kTile; rr += 16) {
+          const int c = lane & 7;
+          if (rr < g.nq_rows) {
+            const uint4 val = lds_v4(stage + rr * 128 + ((c ^ (rr & 7)) << 4));
+            float* orow = a.o_ws + (((size_t)it.split * a.T_q + (g.qrow0 + rr)) * a.H + it.head) * kHeadDim;
+            *reinterpret_cast<uint4*>(orow + ch * 32 + 4 * c) = val;
+          }
         }
+        named_bar_sync(1 + group, kTile);  // the staging area is reused by the next chunk
       }
     }
   }
