@@ -41,8 +41,8 @@ TILE = 128
 # captures summarised in profiles/attn_sm100_stack8.md and
 # profiles/attn_sm100_paged.md; set to None when the kernel changes until it
 # is captured again.
-ATTN_TRAFFIC_BYTES = 392_002_560 + 71_595_776
-PAGED_TRAFFIC_BYTES = 114_754_560 + 5_426_432
+ATTN_TRAFFIC_BYTES = 406_518_528 + 80_945_920
+PAGED_TRAFFIC_BYTES = 114_933_760 + 5_080_576
 
 
 def allowed_pairs(lengths, cands=None):
