@@ -118,19 +118,24 @@ __global__ void __launch_bounds__(256) mf_gather_kernel(MfArgs a) {
   const int c0 = a.cand_offsets[u], C = a.cand_offsets[u + 1] - c0;
   const int first = a.m * a.mb;
   const int row_chunks = a.H * a.d * a.esize / 16;
-  const long long n_items = 4ll * a.mb * row_chunks;
-  for (long long x = blockIdx.y * (long long)blockDim.x + threadIdx.x; x < n_items;
-       x += (long long)gridDim.y * blockDim.x) {
-    const int arr = (int)(x / ((long long)a.mb * row_chunks));
-    const int rem = (int)(x - (long long)arr * a.mb * row_chunks);
-    const int j = rem / row_chunks, ch = rem - j * row_chunks;
+  // a warp copies whole rows (tensor, row) of the microbatch, its lanes
+  // striding over the row's 16-byte chunks: one division per row
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int wr = blockIdx.y * wpb + (threadIdx.x >> 5); wr < 4 * a.mb; wr += gridDim.y * wpb) {
+    const int arr = wr / a.mb;
+    const int j = wr - arr * a.mb;
     const int c = first + j;
     const uint8_t* src = arr == 0 ? a.q : arr == 1 ? a.k : arr == 2 ? a.v : a.u;
     uint8_t* dst = arr == 0 ? a.q_mb : arr == 1 ? a.k_mb : arr == 2 ? a.v_mb : a.u_mb;
     const long long stride = arr == 3 ? a.u_stride : a.qkv_stride;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (c < C) val = *reinterpret_cast<const uint4*>(src + ((size_t)(c0 + c) * stride) * a.esize + (size_t)ch * 16);
-    *reinterpret_cast<uint4*>(dst + ((size_t)u * a.mb + j) * row_chunks * 16 + (size_t)ch * 16) = val;
+    const uint8_t* srow = src + (size_t)(c0 + c) * stride * a.esize;
+    uint8_t* drow = dst + ((size_t)u * a.mb + j) * row_chunks * 16;
+    for (int ch = lane; ch < row_chunks; ch += 32) {
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (c < C) val = *reinterpret_cast<const uint4*>(srow + (size_t)ch * 16);
+      *reinterpret_cast<uint4*>(drow + (size_t)ch * 16) = val;
+    }
   }
   // timestamps: the history, then the rows' (a padding row repeats the latest one)
   const int L = a.cached_lens[u];
