@@ -246,6 +246,9 @@ struct BwdSmem {
   float ds[kBT][kSP];   // ds_ij            [query][key]
   float dst[kBT][kSP];  // ds_ij            [key][query]
   int bk[kBT][kSP];     // time bucket of each pair [query][key]
+  uint4 oct[32];        // octave table of the bucket edges (|dt| + 1 < 2^32)
+  float rts[kMaxBuckets];  // rab_ts
+  float rpw[128];       // rab_pos over the block pair's position differences wbase .. wbase + 126
   float drt[kMaxBuckets];
   long long thr[kMaxBuckets];
   long long tq[kBT], tk[kBT];
@@ -378,7 +381,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   for (int x = tid; x < kMaxBuckets; x += kBwdThreads) {
     sm.thr[x] = tab.thr[x];
     sm.drt[x] = 0.f;
+    sm.rts[x] = x < a.nb ? a.rab_ts[x] : 0.f;
   }
+  if (tid < 32) sm.oct[tid] = make_uint4(tab.oct[tid][0], tab.oct[tid][1], tab.oct[tid][2], tab.oct[tid][3]);
   stage_rows<D>(sm.k, k, j0, n, a.qkv_stride, head);
   stage_rows<D>(sm.v, v, j0, n, a.qkv_stride, head);
   if (tid < kBT) sm.tk[tid] = a.ts[q0 + min(j0 + tid, n - 1)];
@@ -410,6 +415,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     nq.store(sm.q);
     ng.store(sm.g);
     if (tid < kBT) sm.tq[tid] = nts;
+    // rab_pos over the pair's position differences: p_i - p_j - wbase lies in [0, 126]
+    const int wbase = min(i0, hist) - min(j0 + kBT - 1, hist);
+    if (tid < 127) {
+      const int idx = wbase + tid + a.n_max - 1;
+      sm.rpw[tid] = (idx >= 0 && idx < 2 * a.n_max - 1) ? a.rab_pos[idx] : 0.f;
+    }
     __syncthreads();
 
     // S = Q K^T and dP = g V^T on 4 x 4 register tiles
@@ -452,8 +463,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         int bkt = 0;
         if (allowed) {
           const int p_i = min(i, hist), p_j = min(j, hist);
-          bkt = bucket_of_dt(sm.thr, sm.tq[li] - sm.tk[lj]);
-          const float sv = a.alpha * s[r][c] + a.rab_pos[p_i - p_j + a.n_max - 1] + a.rab_ts[bkt];
+          // the octave table below 2^32 (one lookup), the edge search above
+          const long long dt = sm.tq[li] - sm.tk[lj];
+          const unsigned long long xdt = abs_dt_plus1(dt);
+          bkt = xdt < (1ull << 32) ? bucket_oct(sm.oct, (unsigned int)xdt) : bucket_of_dt(sm.thr, dt);
+          const float sv = a.alpha * s[r][c] + sm.rpw[p_i - p_j - wbase] + sm.rts[bkt];
           const float sig = 1.f / (1.f + expf(-sv));
           av = sv * sig * inv_n;
           dsv = dp[r][c] * sig * (1.f + sv * (1.f - sig)) * inv_n;
@@ -472,9 +486,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // bucket only changes near the diagonal), warp-aggregated when all lanes
     // share the bucket.
     if (tid < 127) {
-      const int wbase = min(i0, hist) - min(j0 + kBT - 1, hist);
       const int w = tid;
       float acc = 0.f;
+#pragma unroll 8
       for (int li = 0; li < kBT; ++li) {
         const int i = i0 + li;
         const int pj = min(i, hist) - wbase - w;
