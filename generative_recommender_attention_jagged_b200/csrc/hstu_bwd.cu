@@ -18,11 +18,13 @@
 // stages Q and g in shared memory, forms S = Q K^T and dP = g V^T (4x4
 // register tiles, fp32 FMA), turns them into a and ds, then accumulates
 // d_v += a^T g and d_k += ds^T Q, and adds ds K into d_q with vector atomics
-// (d_q is zeroed first).  Bias gradients are folded per thread, summed in
-// shared memory (a 127-entry window of position differences per block pair, a
-// bucket histogram per CTA) and added to global memory with atomics.  Other
-// head dims take the warp-per-row kernels below, whose warps fold runs of
-// equal bias indices of their own row before the atomics.
+// (d_q is zeroed first).  Bias gradients come from the block pair's ds tile in
+// shared memory: one thread per position difference (127 per pair) sums its
+// pairs and adds the result to d rab_pos with one atomic, and a row walk folds
+// each run of equal time buckets into a per-CTA histogram (warp-aggregated
+// when a warp's lanes share the bucket) that goes to d rab_ts at the end.
+// Other head dims take the warp-per-row kernels below, whose warps fold runs
+// of equal bias indices of their own row before the atomics.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
