@@ -36,6 +36,8 @@ def _need_cuda(name: str, t: Optional[torch.Tensor], dtype=None):
 
 def _rows_view(name: str, t: torch.Tensor, H: int, d: int) -> int:
     """Token stride (elements) of a [T,H,d] (or [T,H*d]) view with packed heads."""
+    if t.numel() == 0:
+        return H * d  # no rows: the layout is immaterial
     if t.dim() == 3:
         ok = t.stride(2) == 1 and t.stride(1) == d
     else:

@@ -144,7 +144,11 @@ struct Common {
 
 int run(const hstu_attn_params* p, const Common& c) {
   if (int rc = check_params(p)) return rc;
-  if (!c.q || !c.k || !c.v || !c.u || !c.q_offsets || !c.ts || !c.rab_pos || !c.rab_ts || !c.out || !c.ws)
+  // arrays indexed by token may be null when there are no tokens (an empty
+  // tensor need not have storage); paged timestamps also cover the prefix
+  const bool rows = p->total_tokens > 0;
+  if ((rows && (!c.q || !c.k || !c.v || !c.u || !c.out)) || (!c.ts && (rows || c.paged)) || !c.q_offsets ||
+      !c.rab_pos || !c.rab_ts || !c.ws)
     return HSTU_ERR_INVALID_ARG;
   if (c.paged && (!c.ts_offsets || !c.cached_lens || !c.page_table || !c.k_pool || !c.v_pool || c.page_size <= 0 ||
                   c.num_pages <= 0 || c.max_pages <= 0))
@@ -339,12 +343,14 @@ int hstu_attn_bwd(const hstu_attn_params* p, const void* q, const void* k, const
                   float* d_rab_pos, float* d_rab_ts, void* workspace, size_t workspace_bytes,
                   hstu_stream_t stream) {
   if (int rc = check_params(p)) return rc;
-  if (!q || !k || !v || !seq_offsets || !timestamps || !rab_pos || !rab_ts || !d_o || !d_q || !d_k || !d_v ||
-      !d_rab_pos || !d_rab_ts || !workspace)
+  // arrays indexed by token may be null when there are no tokens
+  const bool rows = p->total_tokens > 0;
+  if ((rows && (!q || !k || !v || !timestamps || !d_o || !d_q || !d_k || !d_v)) || !seq_offsets || !rab_pos ||
+      !rab_ts || !d_rab_pos || !d_rab_ts || !workspace)
     return HSTU_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, d_o, d_q, d_k, d_v, workspace};
   for (const void* ptr : ptrs)
-    if (!aligned16(ptr)) return HSTU_ERR_ALIGNMENT;
+    if (ptr && !aligned16(ptr)) return HSTU_ERR_ALIGNMENT;
   if (workspace_bytes < sizeof(WsHeader)) return HSTU_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   AttnArgs a;

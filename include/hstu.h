@@ -127,6 +127,8 @@ size_t hstu_attn_workspace_size(const hstu_attn_params* p);
  *   ln_gamma, ln_beta  [H*d] fp32 or NULL (= 1 and = 0)
  *   out            [T, H*d] dtype (fp32 [T,H,d] o with HSTU_F_OUTPUT_RAW_AV)
  *   workspace      device scratch of at least hstu_attn_workspace_size() bytes
+ * With T = 0 the arrays indexed by token (q, k, v, u, timestamps, out) may be
+ * NULL; the call then only checks seq_offsets.
  * Returns HSTU_OK or a negative hstu_status.
  */
 int hstu_attn_fwd(const hstu_attn_params* p, const void* q, const void* k, const void* v,
@@ -276,6 +278,8 @@ int hstu_layer_f2(const hstu_linear_params* p, const void* y, const void* w2, co
  *   d_o         [T, H, d] fp32 contiguous
  *   d_q, d_k, d_v [T, H, d] fp32 contiguous (written)
  *   d_rab_pos   [2*n_max-1] fp32, d_rab_ts [num_ts_buckets] fp32 (zeroed, then summed)
+ * With T = 0 the arrays indexed by token may be NULL (the bias-table
+ * gradients are still zeroed).
  * Device checks as in hstu_attn_fwd (status word in the workspace).
  */
 size_t hstu_attn_bwd_workspace_size(const hstu_attn_params* p);

@@ -39,6 +39,7 @@ def run(b, seed):
     ([200, 65, 128], [70, 0, 1], 2, 64, torch.float32),
     ([64, 130], [64, 3], 1, 128, torch.float32),
     ([40, 9], [5, 0], 1, 48, torch.float32),       # head dim outside the tiled kernel's set
+    ([0, 40, 0, 33, 0], [0, 5, 0, 0, 0], 2, 128, torch.bfloat16),   # empty users
 ])
 def test_gradients_match_oracle(lengths, cands, H, d, dtype):
     rng = np.random.default_rng(sum(lengths))
@@ -61,3 +62,13 @@ def test_unsorted_timestamps_are_reported():
                                 dev(b.timestamps, torch.int64), dev(b.rab_pos, torch.float32),
                                 dev(b.rab_ts, torch.float32), dev(g), n_max=b.n_max, alpha=b.alpha)
     assert hstu.hstu_check_device_error(ws) == -8
+
+
+def test_empty_batch():
+    rng = np.random.default_rng(4)
+    b = synth.jagged_batch([0, 0], 2, 64, 64, rng=rng, dtype=torch.float32)
+    status, got, want = run(b, seed=1)
+    assert status == 0
+    for gv, wv in zip(got, want):
+        assert gv.shape == wv.shape
+        assert not np.any(gv)                   # no pairs: every gradient is zero

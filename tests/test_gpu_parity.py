@@ -139,6 +139,19 @@ def test_work_list_for_few_and_many_users(num_users):
     assert np.abs(o.reshape(o.shape[0], -1)).sum(axis=1).min() > 0   # no row left out of the work list
 
 
+@pytest.mark.parametrize("lengths,cands", [
+    ([0, 300, 0, 129, 0], [0, 40, 0, 0, 0]),   # empty users first, between and last
+    ([0, 0], None),                            # an empty batch (T = 0)
+])
+def test_zero_length_users(lengths, cands):
+    b = small_batch(lengths, cands=cands, n_max=320, seed=3)
+    T = int(sum(lengths))
+    y = run_jagged(b)
+    assert tuple(y.shape) == (T, 4 * 128)
+    if T:
+        assert rel_err(host64(y), oracle.batch_attn(b)) <= BF16_TOL
+
+
 def test_bf16_tensor_core_matches_cuda_core_kernel():
     b = small_batch([400, 131, 77], cands=[50, 0, 3], n_max=512, seed=5)
     o_tc = host64(run_jagged(b, raw_av=True))
