@@ -88,6 +88,26 @@ def test_null_pointers_rejected_on_host(lib):
     assert rc == -1
 
 
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="hands fake device pointers to the library; run only where no GPU can see them")
+def test_empty_batch_accepts_null_token_arrays_on_host(lib):
+    """With T = 0 the token-indexed arrays may be NULL: the host checks pass
+    and the call gets as far as its first CUDA call (which fails here, with no
+    GPU); with T > 0 the same NULLs are an invalid argument."""
+    fake = ctypes.c_void_p(0x1000)
+    for total, want_invalid in ((0, False), (5, True)):
+        p = params(total_tokens=total)
+        args = [None] * 13
+        args[4], args[7], args[8], args[12] = fake, fake, fake, fake  # offsets, rab_pos, rab_ts, workspace
+        rc = lib.hstu_attn_fwd(ctypes.byref(p), *args, 1 << 30, None)
+        assert (rc == -1) == want_invalid, (total, rc)
+        bargs = [None] * 15
+        for i in (3, 6, 7, 12, 13, 14):  # offsets, rab_pos, rab_ts, d_rab_pos, d_rab_ts, workspace
+            bargs[i] = fake
+        rc = lib.hstu_attn_bwd(ctypes.byref(p), *bargs, 1 << 30, None)
+        assert (rc == -1) == want_invalid, (total, rc)
+
+
 def test_misaligned_pointer_rejected_on_host(lib):
     p = params()
     fake = [ctypes.c_void_p(0x1000)] * 13
