@@ -121,6 +121,8 @@ def load() -> ctypes.CDLL:
         fn.restype = ctypes.c_int
     lib.hstu_attn_fwd_static_ws.argtypes = [PP] + [P] * 13
     lib.hstu_attn_fwd_static_ws.restype = ctypes.c_int
+    lib.hstu_static_ws_check_device_error.argtypes = [P]
+    lib.hstu_static_ws_check_device_error.restype = ctypes.c_int
     lib.hstu_attn_bwd_workspace_size.argtypes = [PP]
     lib.hstu_attn_bwd_workspace_size.restype = sz
     lib.hstu_attn_bwd.argtypes = [PP] + [P] * 15 + [sz, P]

@@ -143,21 +143,29 @@ int hstu_attn_fwd(const hstu_attn_params* p, const void* q, const void* k, const
  * memory plan forbids allocation on the request path, or a plug-in whose host
  * runtime owns the allocator).  The pages have no counterpart: this is an
  * interface convenience of this library.  Same arguments and result as
- * hstu_attn_fwd minus workspace/workspace_bytes.  Scratch lives in one
- * 16 MiB device array of the library, held on every GPU that loads it until
- * exit; problems whose hstu_attn_workspace_size() exceeds 16 MiB (about 8,000
- * tokens at H*d = 512) return HSTU_ERR_WORKSPACE before any launch.  All
- * calls share that array: calls whose kernels overlap on the GPU race, so
- * order them (e.g. one stream).  Every call clears the part that must start
- * at zero.  The first call on a device looks up the array's address; make it
- * before any stream capture.  Nothing is allocated.  The device status word
- * sits in that internal array, out of reach of hstu_check_device_error; use
- * hstu_attn_fwd with a workspace of your own when device-side checks matter.
+ * hstu_attn_fwd minus workspace/workspace_bytes (invalid parameters give the
+ * codes hstu_attn_fwd gives).  Scratch lives in one 16 MiB device array of
+ * the library, held on every GPU that loads it until exit; problems whose
+ * hstu_attn_workspace_size() exceeds 16 MiB (about 8,000 tokens at
+ * H*d = 512) return HSTU_ERR_WORKSPACE before any launch.  All calls share
+ * that array: calls whose kernels overlap on the GPU race, so order them
+ * (e.g. one stream).  Every call clears the part that must start at zero.
+ * The first call in a CUDA context looks the array's address up and keeps it
+ * for that context; a call in another context (another device, or the same
+ * device after cudaDeviceReset) looks it up again.  Make each context's first
+ * call before any stream capture.  Nothing is allocated.  The device status
+ * word sits in that internal array: read it with
+ * hstu_static_ws_check_device_error().
  */
 int hstu_attn_fwd_static_ws(const hstu_attn_params* p, const void* q, const void* k, const void* v,
                             const void* u, const int32_t* seq_offsets, const int64_t* timestamps,
                             const int32_t* num_candidates, const float* rab_pos, const float* rab_ts,
                             const float* ln_gamma, const float* ln_beta, void* out, hstu_stream_t stream);
+
+/* Synchronises `stream`, then returns the status word the device wrote during
+ * the last hstu_attn_fwd_static_ws call on the current device (HSTU_OK if
+ * none); HSTU_ERR_CUDA if the array's address cannot be looked up. */
+int hstu_static_ws_check_device_error(hstu_stream_t stream);
 
 /* Bytes of workspace hstu_attn_fwd_paged needs with `num_splits` key splits. */
 size_t hstu_attn_paged_workspace_size(const hstu_attn_params* p, int32_t num_splits);

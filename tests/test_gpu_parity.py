@@ -93,9 +93,8 @@ def test_tiny_fp32_raw_av_and_candidates():
 
 @pytest.mark.parametrize("d", [1, 8, 33, 64, 200])
 def test_fp32_odd_head_dims(d):
-    b = small_batch([9, 17, 3], cands=[0, 4, 0], H=3, d=d, n_max=20, dtype=torch.float32, seed=d)
-    if (3 * d) % 4:
-        pytest.skip("fp32 row stride must be a multiple of 4 elements")
+    # H = 4 keeps the fp32 row stride H*d a multiple of 4 elements for every d
+    b = small_batch([9, 17, 3], cands=[0, 4, 0], H=4, d=d, n_max=20, dtype=torch.float32, seed=d)
     assert rel_err(host64(run_jagged(b)), oracle.batch_attn(b)) <= F32_TOL
 
 
@@ -202,6 +201,114 @@ def test_one_hot_time_bias_selects_exact_buckets():
         _, want_o = oracle.batch_attn(b, want_o=True)
         got = host64(run_jagged(b, raw_av=True))
         assert rel_err(got, want_o) <= 1e-2, bstar
+
+
+# ----------------------------------------------------------------------------
+# time buckets inside the attention kernels: wide gaps, the clamp, small tables
+# ----------------------------------------------------------------------------
+
+def wide_gap_timestamps(rng, lengths, cands=None):
+    """Non-decreasing timestamps whose gaps mix 1-4 s steps, ~600 s steps and
+    jumps of 2^10 .. 2^32 and 2^32 .. 2^52 s, so that every bucket range
+    occurs.  One 32-key chunk then crosses several bucket edges while
+    |dt| + 1 >= 2^32 (the kernels' per-column walk), and pairs far apart reach
+    |dt| + 1 >= e^(0.301*127) ~ 2^55.1, the last bucket (the clamp)."""
+    out = []
+    for i, n in enumerate(lengths):
+        c = 0 if cands is None else int(cands[i])
+        h = int(n) - c
+        m = max(h - 1, 0)
+        kind = rng.choice(4, size=m, p=[0.2, 0.3, 0.2, 0.3])
+        tiny = rng.integers(1, 5, size=m)
+        small = np.maximum(1, np.rint(rng.exponential(600.0, size=m)))
+        medium = np.rint(np.exp2(rng.uniform(10, 32, size=m)))
+        big = np.rint(np.exp2(rng.uniform(32, 52, size=m)))
+        gaps = np.choose(kind, [tiny, small, medium, big]).astype(np.int64)
+        t0 = -(1 << 60) + int(rng.integers(0, 1 << 40))
+        hist = t0 + np.concatenate([np.zeros(1 if h > 0 else 0, np.int64), np.cumsum(gaps)])
+        last = hist[-1] if h > 0 else t0
+        out.append(np.concatenate([hist, np.full(c, last, dtype=np.int64)]))
+    ts = np.concatenate(out)
+    assert np.abs(ts).max() < (1 << 61)  # the library's timestamp range
+    return ts
+
+
+def wide_gap_batch(nb, *, seed, dtype=torch.bfloat16, d=128, H=4):
+    lengths, cands = [1100, 300, 77, 260], [0, 40, 0, 130]
+    b = small_batch(lengths, cands=cands, H=H, d=d, n_max=1200, seed=seed, dtype=dtype,
+                    scale=1.0 if dtype == torch.bfloat16 else 1 / math.sqrt(d))
+    b.timestamps = wide_gap_timestamps(np.random.default_rng(seed + 100), lengths, cands)
+    rng = np.random.default_rng(seed + 200)
+    b.rab_ts = rng.normal(0, 0.5, size=nb).astype(np.float32)   # order-1 entries: a wrong bucket shows
+    return b
+
+
+def test_wide_gap_timestamps_reach_walk_mode_and_clamp():
+    # the inputs below really exercise what they claim (checked on the host
+    # with the oracle's bucket rule)
+    b = wide_gap_batch(128, seed=1)
+    ts, off = b.timestamps, b.seq_offsets
+    lo, hi = int(off[0]), int(off[1])
+    t = ts[lo:hi]
+    dt = t[-1] - t[:64]
+    assert (oracle.ts_bucket(dt) == 127).all()                   # far pairs clamp
+    multi_edge_wide = 0
+    for i in range(200, hi - lo, 37):
+        for c0 in range(0, i - 32, 32):
+            d = t[i] - t[c0:c0 + 32]
+            bk = oracle.ts_bucket(d)
+            if len(set(bk.tolist())) > 2 and (d.min() + 1) >= 2 ** 32:
+                multi_edge_wide += 1
+    assert multi_edge_wide > 20
+
+
+@pytest.mark.parametrize("nb", [1, 16, 100, 128])
+def test_wide_gaps_and_bucket_tables_tensor_core(nb):
+    b = wide_gap_batch(nb, seed=nb)
+    want_y, want_o = oracle.batch_attn(b, want_o=True)
+    o = host64(run_jagged(b, raw_av=True))
+    assert rel_err(o, want_o) <= BF16_TOL
+    y = host64(run_jagged(b))
+    assert rel_err(y, want_y) <= BF16_TOL
+
+
+@pytest.mark.parametrize("nb", [1, 16, 100, 128])
+def test_wide_gaps_and_bucket_tables_cuda_core(nb):
+    b = wide_gap_batch(nb, seed=nb + 7, dtype=torch.float32, d=32, H=2)
+    assert rel_err(host64(run_jagged(b)), oracle.batch_attn(b)) <= F32_TOL
+    b16 = wide_gap_batch(nb, seed=nb + 9)
+    _, want_o = oracle.batch_attn(b16, want_o=True)
+    assert rel_err(host64(run_jagged(b16, raw_av=True, force_simt=True)), want_o) <= 1e-4
+
+
+@pytest.mark.parametrize("nb,bstar", [(128, 127), (128, 100), (128, 70), (128, 44), (100, 99), (16, 15),
+                                      (16, 5), (1, 0)])
+@pytest.mark.parametrize("force_simt", [False, True])
+def test_one_hot_time_bias_wide_gaps(nb, bstar, force_simt):
+    # q = k = 0 and rab_pos = 0: only keys whose (clamped) bucket is bstar
+    # contribute, so one wrong bucket anywhere is a whole v row missing or extra
+    b = wide_gap_batch(nb, seed=3 * bstar + nb)
+    b.q.zero_()
+    b.k.zero_()
+    b.rab_pos[:] = 0
+    b.rab_ts[:] = 0
+    b.rab_ts[bstar] = 4.0
+    _, want_o = oracle.batch_attn(b, want_o=True)
+    assert np.abs(want_o).max() > 0
+    got = host64(run_jagged(b, raw_av=True, force_simt=force_simt))
+    assert rel_err(got, want_o) <= 1e-2
+
+
+def test_paged_wide_gap_timestamps():
+    rng = np.random.default_rng(41)
+    cached, acts, cands = [900, 300], [64, 10], [64, 5]
+    pb = synth.paged_batch(cached, acts, cands, 4, 128, 1100, rng=rng)
+    lengths = [c + a + k for c, a, k in zip(cached, acts, cands)]
+    pb.timestamps = wide_gap_timestamps(np.random.default_rng(42), lengths, cands)
+    pb.rab_ts = np.random.default_rng(43).normal(0, 0.5, size=128).astype(np.float32)
+    want_y, want_o = oracle.batch_paged(pb, want_o=True)
+    assert rel_err(host64(run_paged(pb, raw_av=True, num_splits=2)), want_o) <= BF16_TOL
+    assert rel_err(host64(run_paged(pb, num_splits=2)), want_y) <= BF16_TOL
 
 
 # ----------------------------------------------------------------------------

@@ -213,3 +213,14 @@ def test_mfalcon_rejects_bad_args_on_host(lib):
     assert lib.hstu_mfalcon_fwd(*args(mb=0)) == -1
     assert lib.hstu_mfalcon_fwd(*args(q=None)) == -1
     assert lib.hstu_mfalcon_fwd(*args(q=ctypes.c_void_p(0x1008))) == -3
+
+
+@pytest.mark.parametrize("bad,code", [(dict(batch=0), -1), (dict(num_ts_buckets=129), -2), (dict(head_dim=300), -2),
+                                      (dict(dtype=__import__("torch").bfloat16, num_heads=4, head_dim=3), -3)])
+def test_static_ws_entry_returns_the_workspace_entry_codes(lib, bad, code):
+    # the allocation-free entry point checks the parameters exactly as
+    # hstu_attn_fwd does (no GPU is touched: the checks fail first)
+    p = params(**bad)
+    rc_ws = lib.hstu_attn_fwd(ctypes.byref(p), *([None] * 13), 0, None)
+    rc_static = lib.hstu_attn_fwd_static_ws(ctypes.byref(p), *([None] * 13))
+    assert rc_ws == code and rc_static == code

@@ -395,3 +395,29 @@ def test_f1_block_order():
     w3[:, 2 * hd + d:2 * hd + 2 * d] = 0.0
     _, _, q3, _ = olayer.f1(x, w3, w.b1, H, d)
     assert np.all(q3[:, 1] == 0.0) and np.array_equal(q3[:, 0], q[:, 0])
+
+
+def test_f2_orientation_with_permutation_and_one_hot_weights():
+    # f2 maps y [T, H*d] to x_next [T, d_model] as x_next[t, m] = sum_f y[t, f] W2[f, m] + b2[m].
+    # A permutation W2 (W2[f, m] = 1 iff m = perm[f]) must move feature f of y to
+    # output column perm[f]; the transposed matrix would apply the inverse
+    # permutation instead, which differs for a permutation with no symmetry.
+    rng = np.random.default_rng(11)
+    T, F = 6, 8
+    y = rng.normal(size=(T, F))
+    perm = np.array([3, 0, 6, 1, 7, 2, 5, 4])
+    assert not np.array_equal(perm, np.argsort(perm))      # not its own inverse
+    w2 = np.zeros((F, F))
+    w2[np.arange(F), perm] = 1.0
+    b2 = np.arange(F, dtype=np.float64) * 10.0
+    want = np.empty((T, F))
+    for f in range(F):
+        want[:, perm[f]] = y[:, f]
+    want += b2
+    np.testing.assert_array_equal(olayer.f2(y, w2, b2), want)
+    # a one-hot weight picks one feature into one output column (d_model != H*d)
+    w1hot = np.zeros((F, 3))
+    w1hot[5, 2] = 2.0
+    out = olayer.f2(y, w1hot, np.zeros(3))
+    np.testing.assert_array_equal(out[:, 2], 2.0 * y[:, 5])
+    assert np.all(out[:, :2] == 0.0)
