@@ -75,12 +75,11 @@ constexpr int kTileBytes = kTile * 128 * 2;  // 128 rows x 128 bf16 = 32 KB
 constexpr int kHalfBytes = kTile * 128;      // 128 rows x 64 bf16: one 128B-swizzled box
 constexpr uint32_t kTmemCols = 512;          // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
 constexpr int kHeadDim = 128;
-constexpr int kWin = 384;                    // position-bias window of a 256-row x 128-key block
-constexpr int kWinStride = kWin + 8;         // copies 32 bytes apart: a warp's 16-byte reads hit 8 bank groups
-
+constexpr int kWinChunks = 49;               // elements 0..391 of each copy
+constexpr int kWinLoads = 13;                // producer: R[l + 32 k], k < 13
 struct Meta {
-  long long ts[kTile];          // key timestamps of the tile (the last one repeated past its width)
-  float win[4][kWinStride];     // reversed window of 0.5*rab_pos, four copies shifted by 0..3 floats
+  long long ts[kTile];                       // key timestamps (the last one repeated past the tile's width)
+  uint4 win[kWinChunks][8];                  // 8 copies x 392 bf16, interleaved by 16-byte chunk
 };
 
 struct __align__(1024) Smem {
@@ -91,6 +90,7 @@ struct __align__(1024) Smem {
   long long thr[kMaxBuckets];
   float rab_ts_half[kMaxBuckets];
   uint4 oct[32];
+  uint32_t win_rs[kWinLoads * 16];  // producer scratch: R as 416 bf16
   uint64_t bar_q;
   uint64_t bar_k_full[kStages];
   uint64_t bar_v_full[kStages];
@@ -120,13 +120,6 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-__device__ __forceinline__ float4 lds_f4(const float* p) {
-  float4 r;
-  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-               : "r"(smem_u32(p)));
-  return r;
-}
 
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 r;
@@ -161,14 +154,14 @@ __device__ __forceinline__ uint64_t pk2(float lo, float hi) {
 __device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
@@ -191,14 +184,15 @@ __device__ __forceinline__ void walk_to(Walk& w, long long tj, const long long* 
 // Time-bias modes of a 32-column chunk.
 enum BiasMode { kBiasConst = 0, kBiasEdge = 1, kBiasOct = 2, kBiasWalk = 3 };
 
-// 32 scores of one row: S (fp32 bits) -> P (bf16 pairs).
+// 32 scores of one row: S (fp32 bits, sr[0..31]) -> P (bf16 pairs).  pw[k] is
+// the bf16 pair 0.5 * (rab_pos of column 2k, of column 2k + 1).
 //   kBiasConst: the row's time bucket is the same over the chunk (w.tsb)
 //   kBiasEdge:  one bucket edge: columns before `pos` use tsb_lo, the rest w.tsb
 //   kBiasOct:   every column's bucket from the octave table (|dt| + 1 < 2^32)
 //   kBiasWalk:  per-column walk over the bucket edges (wider gaps)
 // MASK zeroes the columns past climit.
 template <int MODE, bool MASK, bool PRECISE>
-__device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&pk)[16], const float* wp,
+__device__ __forceinline__ void silu_chunk(const uint32_t* sr, const uint32_t (&pw)[16], uint32_t (&pk)[16],
                                            const long long* ts, int col0, int climit, int pos, float tsb_lo,
                                            float alpha_half, Walk& w, const long long* thr, const float* rts,
                                            const uint4* oct) {
@@ -220,37 +214,31 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&
     }
   };
 #pragma unroll
-  for (int c4 = 0; c4 < 8; ++c4) {
-    const float4 w4 = lds_f4(wp + col0 + 4 * c4);
-#pragma unroll
-    for (int hlf = 0; hlf < 2; ++hlf) {
-      const int c = 4 * c4 + 2 * hlf;
-      uint64_t bias2 = hlf == 0 ? pk2(w4.x, w4.y) : pk2(w4.z, w4.w);
-      if constexpr (MODE == kBiasConst) {
-        bias2 = add2(bias2, tsb2);
-      } else {
-        const float t0 = ts_bias(col0 + c);
-        const float t1 = ts_bias(col0 + c + 1);
-        bias2 = add2(bias2, pk2(t0, t1));
-      }
-      const uint64_t h2 = fma2(pk2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), ah2, bias2);
-      float h0, h1;
-      upk2(h2, h0, h1);
+  for (int c = 0; c < 32; c += 2) {
+    uint64_t tb2 = tsb2;
+    if constexpr (MODE != kBiasConst) tb2 = pk2(ts_bias(col0 + c), ts_bias(col0 + c + 1));
+    const uint64_t h2 = fma2(pk2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), ah2, tb2);
+    float h0, h1;
+    upk2(h2, h0, h1);
+    const uint32_t pb = pw[c >> 1];
+    if constexpr (PRECISE) {
+      // fp32: P = hb (1 + tanh hb), one MUFU tanh per score, rounded once to bf16
+      h0 += __uint_as_float(pb << 16);
+      h1 += __uint_as_float(pb & 0xFFFF0000u);
       if constexpr (MASK) {  // SiLU(0) = 0 exactly: masking hb masks P
         h0 = (col0 + c <= climit) ? h0 : 0.f;
         h1 = (col0 + c + 1 <= climit) ? h1 : 0.f;
       }
-      if constexpr (PRECISE) {
-        // fp32: P = hb (1 + tanh hb), one MUFU tanh per score, rounded once to bf16
-        const uint64_t p2 = fma2(pk2(h0, h1), pk2(tanh_approx(h0), tanh_approx(h1)), pk2(h0, h1));
-        float p0, p1;
-        upk2(p2, p0, p1);
-        pk[c >> 1] = pack_bf16x2(p0, p1);
-      } else {
-        // packed bf16: one MUFU tanh per two scores; P = hb (1 + tanh hb) as one bf16x2 FMA
-        const uint32_t hb = pack_bf16x2(h0, h1);
-        pk[c >> 1] = fma_bf16x2(hb, tanh_bf16x2(hb), hb);
-      }
+      const uint64_t p2 = fma2(pk2(h0, h1), pk2(tanh_approx(h0), tanh_approx(h1)), pk2(h0, h1));
+      float p0, p1;
+      upk2(p2, p0, p1);
+      pk[c >> 1] = pack_bf16x2(p0, p1);
+    } else {
+      // packed bf16: one MUFU tanh per two scores; P = hb (1 + tanh hb) as one bf16x2 FMA
+      uint32_t hb = add_bf16x2(pack_bf16x2(h0, h1), pb);
+      if constexpr (MASK)
+        hb &= (col0 + c <= climit ? 0x0000FFFFu : 0u) | (col0 + c + 1 <= climit ? 0xFFFF0000u : 0u);
+      pk[c >> 1] = fma_bf16x2(hb, tanh_bf16x2(hb), hb);
     }
   }
   if constexpr (MODE == kBiasOct) {  // the walk state continues from the chunk's last column
@@ -261,18 +249,55 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&sr)[32], uint32_t (&
 }
 
 template <bool MASK, bool PRECISE>
-__device__ __forceinline__ void silu_chunk_mode(int mode, const uint32_t (&sr)[32], uint32_t (&pk)[16],
-                                                const float* wp, const long long* ts, int col0, int climit,
+__device__ __forceinline__ void silu_chunk_mode(int mode, const uint32_t* sr, const uint32_t (&pw)[16],
+                                                uint32_t (&pk)[16], const long long* ts, int col0, int climit,
                                                 int pos, float tsb_lo, float alpha_half, Walk& w,
                                                 const long long* thr, const float* rts, const uint4* oct) {
   if (mode == kBiasConst)
-    silu_chunk<kBiasConst, MASK, PRECISE>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+    silu_chunk<kBiasConst, MASK, PRECISE>(sr, pw, pk, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
   else if (mode == kBiasEdge)
-    silu_chunk<kBiasEdge, MASK, PRECISE>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+    silu_chunk<kBiasEdge, MASK, PRECISE>(sr, pw, pk, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
   else if (mode == kBiasOct)
-    silu_chunk<kBiasOct, MASK, PRECISE>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+    silu_chunk<kBiasOct, MASK, PRECISE>(sr, pw, pk, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
   else
-    silu_chunk<kBiasWalk, MASK, PRECISE>(sr, pk, wp, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+    silu_chunk<kBiasWalk, MASK, PRECISE>(sr, pw, pk, ts, col0, climit, pos, tsb_lo, alpha_half, w, thr, rts, oct);
+}
+
+// Time-bias mode of the chunk starting at col0 for this row, decided by the
+// warp (the walk state describes the last column processed so far).  May step
+// the walk over one edge (edge mode); returns the mode, the edge column `pos`
+// and the bias before the edge `tsb_lo`.
+__device__ __forceinline__ int chunk_mode(Walk& w, const long long* ts, int col0, int climit,
+                                          const long long* thr, const float* rts, int& pos, float& tsb_lo) {
+  const int col_last = min(col0 + 31, climit);
+  const bool none = col_last < col0;                    // chunk fully masked for this row
+  const long long t_last = ts[max(col_last, 0)];
+  const bool uni = none || t_last <= w.tlim;            // no bucket edge in the chunk
+  int mode = kBiasConst;
+  pos = col0 + 32;
+  tsb_lo = w.tsb;
+  if (!__all_sync(~0u, uni)) {
+    const long long tlim2 = w.b > 0 ? w.t_i + 1 - thr[w.b - 1] : LLONG_MIN;
+    const bool one = uni || t_last <= tlim2;              // at most one edge in the chunk
+    // octave mode needs |dt| + 1 < 2^32 at the chunk's first allowed column
+    const bool narrow = uni || (w.t_i + 1 - ts[col0]) < (1ll << 32);
+    if (__all_sync(~0u, one)) {
+      mode = kBiasEdge;
+      if (!uni) {
+        // first column of the chunk past the edge (timestamps are sorted)
+        pos = col0;
+#pragma unroll
+        for (int step = 16; step >= 1; step >>= 1)
+          if (ts[pos + step - 1] <= w.tlim) pos += step;
+        --w.b;
+        w.tlim = tlim2;
+        w.tsb = rts[w.b];
+      }
+    } else {
+      mode = __all_sync(~0u, narrow) ? kBiasOct : kBiasWalk;
+    }
+  }
+  return mode;
 }
 
 template <bool PRECISE>
@@ -370,7 +395,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // registers one tile ahead, so its global-load latency hides behind the
     // wait for a free stage.  Lane l holds timestamps of columns l + 32k and
     // window entries x = l + 32k - 3 (x in [-3, 384)).
-    constexpr int kWinLoads = (kWin + 3 + 31) / 32;
     long long mts[4];
     float mwin[kWinLoads];
     auto load_meta = [&](int t) {
@@ -378,10 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       key_tile(gA, tb + t, k0, width);
 #pragma unroll
       for (int k = 0; k < 4; ++k) mts[k] = a.ts[gA.tso + k0 + min(lane + 32 * k, width - 1)];
-      const int wb = prmin - k0 - 127 + a.n_max - 1;  // rab_pos index of window entry x = 0
+      const int g0 = prmin + 255 - k0 + a.n_max - 1;  // rab_pos index of R[0]
 #pragma unroll
       for (int k = 0; k < kWinLoads; ++k) {
-        const int idx = wb + lane + 32 * k - 3;
+        const int idx = g0 - (lane + 32 * k);
         mwin[k] = (idx >= 0 && idx < n_rab) ? 0.5f * __ldg(a.rab_pos + idx) : 0.f;
       }
     };
@@ -461,14 +485,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       Meta& m = sm.meta[s];
 #pragma unroll
       for (int k = 0; k < 4; ++k) m.ts[lane + 32 * k] = mts[k];
+      __syncwarp();
+      uint16_t* rs16 = reinterpret_cast<uint16_t*>(sm.win_rs);
 #pragma unroll
-      for (int k = 0; k < kWinLoads; ++k) {
-        const int x = lane + 32 * k - 3;  // copy p, entry z holds window entry 383 - z - p
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const int z = (kWin - 1) - x - p;
-          if (z >= 0 && z < kWin) m.win[p][z] = mwin[k];
-        }
+      for (int k = 0; k < kWinLoads; ++k) rs16[lane + 32 * k] = __bfloat16_as_ushort(__float2bfloat16_rn(mwin[k]));
+      __syncwarp();
+      for (int q = lane; q < kWinChunks * 8; q += 32) {
+        const int f = q >> 3, p = q & 7;
+        const int wb = 4 * f + (p >> 1);
+        const uint32_t sh = 16u * (p & 1);
+        const uint32_t x0 = sm.win_rs[wb], x1 = sm.win_rs[wb + 1], x2 = sm.win_rs[wb + 2],
+                       x3 = sm.win_rs[wb + 3], x4 = sm.win_rs[wb + 4];
+        m.win[f][p] = make_uint4(__funnelshift_r(x0, x1, sh), __funnelshift_r(x1, x2, sh),
+                                 __funnelshift_r(x2, x3, sh), __funnelshift_r(x3, x4, sh));
       }
       mbar_arrive(&sm.bar_meta_full[s]);
       if (t + 1 < cT) load_meta(t + 1);
@@ -560,9 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = min(g.qs + r, g.n - 1);  // rows past the user repeat its last row (discarded)
     const int jmax = i < g.h ? i : g.h - 1;
     const int pr = min(i, g.h);
-    const int y0 = 256 - (pr - prmin);     // window entry of column 0 (reversed window)
-    const int wcopy = y0 & 3;
-    const int woff = y0 - wcopy;
+    const int zb = prmin + 255 - pr;       // window element of column 0
     const float alpha_half = 0.5f * a.alpha;
     const uint32_t s_tmem = tmem + lane_base + x * 128;
     Walk w;
@@ -588,48 +615,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         w.tsb = sm.rab_ts_half[w.b];
       }
       const bool need_mask = !__all_sync(~0u, climit >= kTile - 1);
-      const float* wp = &m.win[wcopy][woff];
 #pragma unroll 1
       for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
         uint32_t sr[32];
         tmem_ld32(s_tmem + ch * 32, sr);
-        // time-bias mode of this chunk (decided while the TMEM load is in flight):
-        // the walk state always describes the last column processed so far
         const int col0 = ch * 32;
-        const int col_last = min(col0 + 31, climit);
-        const bool none = col_last < col0;                    // chunk fully masked for this row
-        const long long t_last = m.ts[max(col_last, 0)];
-        const bool uni = none || t_last <= w.tlim;            // no bucket edge in the chunk
-        int mode = kBiasConst, pos = col0 + 32;
-        float tsb_lo = w.tsb;
-        if (!__all_sync(~0u, uni)) {
-          const long long tlim2 = w.b > 0 ? w.t_i + 1 - sm.thr[w.b - 1] : LLONG_MIN;
-          const bool one = uni || t_last <= tlim2;              // at most one edge in the chunk
-          // octave mode needs |dt| + 1 < 2^32 at the chunk's first allowed column
-          const bool narrow = uni || (w.t_i + 1 - m.ts[col0]) < (1ll << 32);
-          if (__all_sync(~0u, one)) {
-            mode = kBiasEdge;
-            if (!uni) {
-              // first column of the chunk past the edge (timestamps are sorted)
-              pos = col0;
+        int pos;
+        float tsb_lo;
+        const int mode = chunk_mode(w, m.ts, col0, climit, sm.thr, sm.rab_ts_half, pos, tsb_lo);
+        const int z0 = zb + col0;
+        const uint32_t wbase = smem_u32(&m.win[z0 >> 3][z0 & 7]);
+        uint32_t pw[16];
 #pragma unroll
-              for (int step = 16; step >= 1; step >>= 1)
-                if (m.ts[pos + step - 1] <= w.tlim) pos += step;
-              --w.b;
-              w.tlim = tlim2;
-              w.tsb = sm.rab_ts_half[w.b];
-            }
-          } else {
-            mode = __all_sync(~0u, narrow) ? kBiasOct : kBiasWalk;
-          }
+        for (int k = 0; k < 4; ++k) {
+          const uint4 v4 = lds_v4(wbase + k * 8 * 16);
+          pw[4 * k] = v4.x;
+          pw[4 * k + 1] = v4.y;
+          pw[4 * k + 2] = v4.z;
+          pw[4 * k + 3] = v4.w;
         }
         tmem_wait_ld(sr);
         uint32_t pk[16];
         if (need_mask)
-          silu_chunk_mode<true, PRECISE>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w,
+          silu_chunk_mode<true, PRECISE>(mode, sr, pw, pk, m.ts, col0, climit, pos, tsb_lo, alpha_half, w,
                                          sm.thr, sm.rab_ts_half, sm.oct);
         else
-          silu_chunk_mode<false, PRECISE>(mode, sr, pk, wp, m.ts, col0, climit, pos, tsb_lo, alpha_half, w,
+          silu_chunk_mode<false, PRECISE>(mode, sr, pw, pk, m.ts, col0, climit, pos, tsb_lo, alpha_half, w,
                                           sm.thr, sm.rab_ts_half, sm.oct);
         // P of this chunk packs into the warpgroup's own (already read) S columns:
         // keys 0-63 at columns 0-31, keys 64-127 at columns 64-95
@@ -644,8 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ew_all(mbar_wait(&sm.bar_o_full[x], 0, abort_flag, a.hdr, 7), group);
       tc_fence_after();
     }
-    // with no key tile nothing waited for Q; it lands in the staging area below
-    if (ok && cT == 0) ok = ew_all(mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 7), group);
+    // a tile with no key tile of this split (the whole item, or only this
+    // tile when the other has some) issued no GEMM, so nothing waited for its
+    // Q copy; that copy lands in the staging area used below
+    if (ok && cnt == 0 && exists) ok = ew_all(mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 7), group);
     if (ok && exists) {
       // O of this warpgroup's 64 columns goes out through shared memory, 32
       // columns at a time: its half of the tile's Q buffer (free once the
