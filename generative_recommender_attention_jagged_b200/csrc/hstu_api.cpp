@@ -105,15 +105,25 @@ bool use_tensor_cores(const hstu_attn_params* p) {
   return !(p->flags & HSTU_F_FORCE_SIMT) && p->dtype == HSTU_DT_BF16 && p->head_dim == 128 && device_is_sm100();
 }
 
+// Query tiles per tensor-core work item.  A paged call whose users have on
+// average at most one tile of new rows (incremental serving: a few actions and
+// candidates against a long cached prefix) runs the one-tile kernel, which
+// keeps all its warps on that tile and double-buffers S; everything else runs
+// the two-tile kernel, which reads each K/V tile once for 256 query rows.
+int item_tiles_for(const hstu_attn_params* p, bool paged) {
+  return paged && (long long)p->total_tokens <= (long long)kTile * p->batch ? 1 : 2;
+}
+
 struct Layout {
   size_t items_off, o_off, total;
   int max_items;
 };
 
-Layout layout_for(const hstu_attn_params* p, int splits, bool tc) {
+Layout layout_for(const hstu_attn_params* p, int splits, bool tc, int item_tiles) {
   Layout l;
   const long long T = p->total_tokens;
-  const long long qtiles = (T + kItemRows - 1) / kItemRows + p->batch;  // sum_u ceil(n_u/256) <= T/256 + B
+  const long long rows = (long long)item_tiles * kTile;
+  const long long qtiles = (T + rows - 1) / rows + p->batch;  // sum_u ceil(n_u/rows) <= T/rows + B
   const long long items = tc ? qtiles * p->num_heads * splits : 0;
   l.max_items = (int)items;
   l.items_off = sizeof(WsHeader);
@@ -160,7 +170,8 @@ int run(const hstu_attn_params* p, const Common& c) {
   const bool tc = use_tensor_cores(p);
   // tensor-core path: whole pages land as 1024-byte-aligned swizzled boxes
   if (tc && c.paged && (c.page_size < 8 || c.page_size > kTile || kTile % c.page_size)) return HSTU_ERR_UNSUPPORTED;
-  const Layout l = layout_for(p, tc ? c.splits : 1, tc);
+  const int item_tiles = item_tiles_for(p, c.paged);
+  const Layout l = layout_for(p, tc ? c.splits : 1, tc, item_tiles);
   if (c.ws_bytes < l.total) return HSTU_ERR_WORKSPACE;
 
   uint32_t stages = p->flags & (HSTU_F_STAGE_PLAN | HSTU_F_STAGE_ATTN | HSTU_F_STAGE_EPILOGUE);
@@ -184,6 +195,7 @@ int run(const hstu_attn_params* p, const Common& c) {
   a.num_pages = c.num_pages;
   a.max_pages = c.max_pages;
   a.max_items = l.max_items;
+  a.item_tiles = item_tiles;
   a.out_raw = (p->flags & HSTU_F_OUTPUT_RAW_AV) ? 1 : 0;
   a.self_term = tc ? 1 : 0;
   a.out_bf16 = p->dtype == HSTU_DT_BF16 ? 1 : 0;
@@ -229,7 +241,8 @@ int run(const hstu_attn_params* p, const Common& c) {
       if (c.paged && (!encode_pool(&tkp, c.k_pool, c.num_pages, a.H, c.page_size, a.d) ||
                       !encode_pool(&tvp, c.v_pool, c.num_pages, a.H, c.page_size, a.d)))
         return HSTU_ERR_CUDA;
-      e = launch_attn_sm100(a, thr, tq, tk, tv, tkp, tvp, c.stream);
+      e = item_tiles == 1 ? launch_attn_sm100_single(a, thr, tq, tk, tv, tkp, tvp, c.stream)
+                          : launch_attn_sm100(a, thr, tq, tk, tv, tkp, tvp, c.stream);
     } else {
       e = launch_attn_simt(a, thr, c.stream);
     }
@@ -247,13 +260,13 @@ extern "C" {
 
 size_t hstu_attn_workspace_size(const hstu_attn_params* p) {
   if (check_params(p) != HSTU_OK) return 0;
-  return layout_for(p, 1, use_tensor_cores(p)).total;
+  return layout_for(p, 1, use_tensor_cores(p), item_tiles_for(p, false)).total;
 }
 
 size_t hstu_attn_paged_workspace_size(const hstu_attn_params* p, int32_t num_splits) {
   if (check_params(p) != HSTU_OK || num_splits < 1 || num_splits > kMaxSplits) return 0;
   const bool tc = use_tensor_cores(p);
-  return layout_for(p, tc ? num_splits : 1, tc).total;
+  return layout_for(p, tc ? num_splits : 1, tc, item_tiles_for(p, true)).total;
 }
 
 int32_t hstu_attn_paged_default_splits(const hstu_attn_params* p, int32_t max_cached_len) {
@@ -261,7 +274,8 @@ int32_t hstu_attn_paged_default_splits(const hstu_attn_params* p, int32_t max_ca
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // work items before splitting: every user has at least one block of query rows
-  const long long qblocks = std::max<long long>(p->batch, (p->total_tokens + kItemRows - 1) / kItemRows);
+  const long long rows = (long long)item_tiles_for(p, true) * kTile;
+  const long long qblocks = std::max<long long>(p->batch, (p->total_tokens + rows - 1) / rows);
   const long long units = std::max<long long>(1, qblocks * p->num_heads);
   const long long key_tiles = std::max(1, (max_cached_len + kTile - 1) / kTile);
   long long s = std::max<long long>(1, sms / units);  // fill one wave of CTAs, not more

@@ -10,7 +10,7 @@ namespace hstu {
 
 constexpr int kMaxBuckets = 128;   // rab_ts entries supported
 constexpr int kTile = 128;         // query rows / key rows per tensor-core tile
-constexpr int kItemRows = 256;     // query rows per tensor-core work item (two tiles)
+constexpr int kItemRows = 256;     // query rows per work item of the two-tile kernel
 constexpr int kMaxSplits = 64;
 
 // Bucket edges: thr[b] = smallest integer x with ln(x) >= 0.301*b, for
@@ -45,10 +45,10 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header size");
 
-// Work item: one (user, block of kItemRows query rows, head, key split).
+// Work item: one (user, block of item_tiles * kTile query rows, head, key split).
 struct WorkItem {
   int32_t user;
-  int32_t qtile;  // index of the kItemRows-row block inside the user's query rows
+  int32_t qtile;  // index of the block of query rows inside the user's query rows
   int32_t head;
   int32_t split;
 };
@@ -65,6 +65,7 @@ struct AttnArgs {
   int32_t num_splits;
   int32_t page_size, num_pages, max_pages;
   int32_t max_items;
+  int32_t item_tiles;   // query tiles per work item: 2 (two-tile kernel) or 1 (one-tile kernel)
   int32_t out_raw;      // write o (fp32 [T,H,d]) instead of y
   int32_t self_term;    // epilogue adds a_ii v_i for candidate rows (tensor-core path)
   int32_t out_bf16;     // out dtype
@@ -117,6 +118,12 @@ cudaError_t launch_attn_sm100(const AttnArgs& a, const BucketTable& thr, const C
                               const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                               const CUtensorMap& tm_kpool, const CUtensorMap& tm_vpool,
                               cudaStream_t s);
+// One query tile per CTA (items of kTile rows), S double-buffered in tensor
+// memory: for calls whose users have few query rows against long key ranges
+// (the paged incremental mode).
+cudaError_t launch_attn_sm100_single(const AttnArgs& a, const BucketTable& thr, const CUtensorMap& tm_q,
+                                     const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                     const CUtensorMap& tm_kpool, const CUtensorMap& tm_vpool, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnArgs& a, const BucketTable& thr, cudaStream_t s);
 
 // Backward of the attention core on CUDA cores (hstu_bwd.cu); gradients fp32,

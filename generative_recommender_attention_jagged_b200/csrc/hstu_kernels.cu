@@ -52,7 +52,7 @@ __device__ __forceinline__ int check_user(const AttnArgs& a, int u, int& n, int&
   return ok;
 }
 
-// work list: per user, blocks of kItemRows query rows, each expanded to
+// work list: per user, blocks of item_tiles * kTile query rows, each expanded to
 // H heads x num_splits splits; counting sort by cost (key tiles per split).
 // The block's threads form min(B, 256) groups; group g takes users g, g + G, ..
 // and its threads share each user's query blocks, so a batch of a few long
@@ -62,7 +62,8 @@ __device__ void build_schedule(const AttnArgs& a, int* hist, int* start) {
   for (int x = tid; x < kCostBins; x += blockDim.x) hist[x] = 0;
   __syncthreads();
   const int per = a.H * a.num_splits;
-  constexpr int tiles_per_item = kItemRows / kTile;
+  const int tiles_per_item = a.item_tiles;
+  const int item_rows = tiles_per_item * kTile;
   struct UserGeom {
     int L, n, h, nq;
   };
@@ -88,7 +89,7 @@ __device__ void build_schedule(const AttnArgs& a, int* hist, int* start) {
   if (active)
     for (int u = grp; u < a.B; u += groups) {
       const UserGeom g = user_geom(u);
-      for (int m = sub; m < ceil_div(g.nq, kItemRows); m += group_size) atomicAdd(&hist[cost_of(g, m)], per);
+      for (int m = sub; m < ceil_div(g.nq, item_rows); m += group_size) atomicAdd(&hist[cost_of(g, m)], per);
     }
   __syncthreads();
   // start[c] = number of items with a cost above c (descending order): thread t
@@ -123,7 +124,7 @@ __device__ void build_schedule(const AttnArgs& a, int* hist, int* start) {
   if (active)
     for (int u = grp; u < a.B; u += groups) {
       const UserGeom g = user_geom(u);
-      for (int m = sub; m < ceil_div(g.nq, kItemRows); m += group_size) {
+      for (int m = sub; m < ceil_div(g.nq, item_rows); m += group_size) {
         const int pos = atomicAdd(&start[cost_of(g, m)], per);
         for (int h = 0; h < a.H; ++h)
           for (int s = 0; s < a.num_splits; ++s) {
