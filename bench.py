@@ -39,13 +39,13 @@ TILE = 128
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention-kernel launch
 # (layer 0 of the 8-layer stack workload) and of one paged attention launch,
 # each from a single-launch capture on a B200:
-#   ncu --set full --clock-control none -k regex:attn_sm100 -s 2 -c 1 \
-#       python bench.py --steps 1 --warmup 3 --only stack --e2e-steps 0 --layers 1
-#   ncu --set full --clock-control none -k regex:attn_sm100 -s 30 -c 1 \
-#       python bench.py --paged-only --steps 3 --warmup 3
+#   ncu --set full --clock-control none -k regex:attn_sm100_kernel -s 2 -c 1 \
+#       python bench.py --only stack --steps 2 --warmup 3 --e2e-steps 0 --no-cpu-baseline --layers 1
+#   ncu --set full --clock-control none -k regex:attn_sm100_single -s 10 -c 1 \
+#       python bench.py --only paged --steps 3 --warmup 3
 # None whenever the kernel has changed since its counters were taken.
-ATTN_TRAFFIC_BYTES = None
-PAGED_TRAFFIC_BYTES = None
+ATTN_TRAFFIC_BYTES = 406_045_696 + 76_942_848
+PAGED_TRAFFIC_BYTES = 115_100_672 + 5_167_104
 
 
 def allowed_pairs(lengths, cands=None):
@@ -787,7 +787,7 @@ def run_paged_bench(args, device):
                         "+64 candidates, 8 layers (separate pools), H=4, d=128, N_max=8320",
             "ms_per_layer": round(ms_layer, 4), "new_tokens_per_s": round(T / (ms_layer * 1e-3), 1),
             "splits": splits,
-            "roofline": {"kernel": "attn_sm100_kernel (paged)", "bound": "hbm", "achieved": round(achieved, 1),
+            "roofline": {"kernel": "attn_sm100_single_kernel (paged)", "bound": "hbm", "achieved": round(achieved, 1),
                          "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                          "frac": round(achieved / float(peaks["hbm_gbs"]), 4),
                          "peak_source": f"{kind} hbm_gbs", "bytes_per_launch": alg_bytes,
