@@ -692,7 +692,7 @@ def run_layer_bench(args, device):
                           "f2": round(float(np.median(f2_ms)), 4),
                           "plan+epilogue": round(float(np.median([a + c for a, c in zip(part(1, 2), part(3, 4))])), 4)},
             "roofline": tensor_roofline("attn_sm100_kernel", attn_flops, attn_ms, clk),
-            "roofline_f1": tensor_roofline("gemm_bias_act_kernel (f1)", f1_flops, f1_ms, clk),
+            "roofline_f1": tensor_roofline("gemm_pair_kernel (f1)", f1_flops, f1_ms, clk),
             "clocks": clk, "gpu_launches_per_layer": 5, "l2": "two alternating input sets"}
     if not args.no_cpu_baseline:
         b0 = synth.workload_attention("layer_bf16")
@@ -852,9 +852,9 @@ def run_glue_bench(args, device):
             "cublaslt": {"f1_ms": round(f1_lib, 4), "f2_ms": round(f2_lib, 4),
                          "f1_tflops": round(tf(f1_flops, f1_lib), 1), "f2_tflops": round(tf(f2_flops, f2_lib), 1),
                          "note": "cuBLASLt GEMM, bias in its epilogue, separate in-place SiLU pass for f1"},
-            "roofline": tensor_roofline("gemm_bias_act_kernel (f1: bias + SiLU in the epilogue)", f1_flops,
+            "roofline": tensor_roofline("gemm_pair_kernel (f1: bias + SiLU in the epilogue)", f1_flops,
                                         *samples["f1"]),
-            "roofline_f2": tensor_roofline("f2 = y W2 + b2", f2_flops, *samples["f2"])}
+            "roofline_f2": tensor_roofline("gemm_pair_kernel (f2 = y W2 + b2)", f2_flops, *samples["f2"])}
 
 
 def run_mfalcon_bench(args, device):

@@ -1,21 +1,28 @@
-// out = act(x W + bias) on the sm_100a tensor cores, bias and activation in
-// the GEMM's own epilogue (the layer's f1 with SiLU, f2 without).
+// out = act(x W + bias) on a pair of SMs (tcgen05 cta_group::2), bias and
+// activation in the epilogue: the layer's f1 (SiLU) and f2 projections.
 //
-// x [T, K] bf16 (row stride x_stride), W [K, N] bf16 row-major, out [T, N] bf16.
-// Output tile 128 x 256, K in blocks of 64:
-//   A = x tile  (128 rows x 64 K, K-major, 128B swizzle: one TMA box)
-//   B = W block (64 K rows x 256 N, N-major: four TMA boxes of 64 N columns)
-//   D = fp32 accumulator in tensor memory, two 256-column buffers so that the
-//       epilogue of one tile overlaps the MMAs of the next
-// Persistent CTAs walk the tiles (row-block major, so CTAs running at the
-// same time share x rows in L2).  Warp roles (320 threads): warp 0 TMA
-// producer, warp 1 MMA issuer and tensor-memory owner, warps 2-9 epilogue
-// (thread = output row = TMEM lane, two warps per lane quarter splitting the
-// columns): tcgen05.ld 32 columns at a time, add the
-// fp32 bias, SiLU as h + h tanh(h) with h = x/2 (one MUFU op per element),
-// round to bf16, 16-byte stores of the thread's own row.  Rows past T are
-// zero-filled by TMA on the way in and not stored on the way out.  Every wait
-// is bounded and reports HSTU_ERR_TIMEOUT through the workspace status word.
+// Why a pair: a single-SM 128 x 256 tile reads its A and B operands from
+// shared memory at 96 B/clk while TMA writes the next stages at about the
+// same rate, more than the SM's shared memory delivers, so the tensor core
+// waits.  Two CTAs of a cluster share one 256 x 256 output tile: each holds
+// its own 128 rows of x and half (128 columns) of the W block, the MMA
+// (M = 256, N = 256, K = 16, issued by the even CTA) reads both CTAs' shared
+// memory, and each SM then reads 64 B/clk of operands and takes 64 B/clk of
+// TMA writes.  Each CTA's accumulator is its 128 rows x 256 columns in its
+// own tensor memory (two buffers: the epilogue of one tile overlaps the MMAs
+// of the next).
+//
+// Roles (320 threads per CTA): warp 0 TMA producer (both CTAs load their own
+// x rows and W half; the bytes complete on the even CTA's barrier), warp 1
+// MMA issuer (even CTA only) and tensor-memory owner (both CTAs allocate
+// collectively), warps 2-9 epilogue (thread = output row, two warps per lane
+// quarter splitting the 256 columns): tcgen05.ld, fp32 bias, SiLU as
+// h + h tanh h with h = x / 2, bf16 into a 128B-swizzled staging tile that
+// one thread stores with TMA (whole 128-byte row segments).  The
+// odd CTA's epilogue frees an accumulator by a remote arrive on the even
+// CTA's barrier.  Every wait is bounded; whatever happens, both CTAs meet at
+// a cluster barrier before tensor memory is freed and the CTAs exit, so
+// neither leaves while the other's MMAs may still read its shared memory.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -29,29 +36,36 @@
 namespace hstu {
 namespace {
 
-constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
-constexpr int kXStage = kBM * kBK * 2;         // 16 KB
-constexpr int kWChunk = kBK * 64 * 2;          // 64 K rows x 64 N columns = 8 KB
-constexpr int kWStage = kWChunk * (kBN / 64);  // 32 KB
-constexpr int kEpiWarps = 8;                  // two per TMEM lane quarter: each takes half the columns
-constexpr int kGemmThreads = 32 * (2 + kEpiWarps);
-constexpr uint32_t kAccCols = kBN;             // one fp32 accumulator: 256 columns
+constexpr int kBM = 128;                          // rows per CTA (256 per pair)
+constexpr int kBN = 256;                          // columns per pair tile (128 of W per CTA)
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kXStage = kBM * kBK * 2;            // 16 KB
+constexpr int kWChunk = kBK * 64 * 2;             // 64 K rows x 64 N columns = 8 KB
+constexpr int kWStage = kWChunk * (kBN / 2 / 64); // this CTA's 128 columns: 16 KB
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr uint32_t kAccCols = kBN;                // one fp32 accumulator: 256 columns
+constexpr uint32_t kPeerMask = 0xFEFFFFFFu;       // clears the CTA-rank bit of a shared::cluster address
 
-struct __align__(1024) GemmSmem {
+constexpr int kOutBox = kBM * 128;               // 128 rows x 64 bf16 columns of output: 16 KB
+
+struct __align__(1024) Smem2 {
   uint8_t x[kStages][kXStage];
   uint8_t w[kStages][kWStage];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
-  uint64_t done;
+  uint8_t out[kBN / 64][kOutBox];  // this CTA's 128 x 256 bf16 tile, four 128B-swizzled TMA boxes
+  uint64_t full[kStages];       // even CTA: both CTAs' bytes of the stage landed
+  uint64_t empty[kStages];      // both CTAs: the MMAs that read the stage completed
+  uint64_t acc_full[2];         // both CTAs: accumulator b holds a finished tile
+  uint64_t acc_empty[2];        // even CTA: both CTAs' epilogues read accumulator b
+  uint64_t done;                // both CTAs: every MMA completed
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t kGemmSmem = sizeof(GemmSmem) + 1024;
-static_assert(kGemmSmem <= 227 * 1024, "shared memory budget");
+constexpr size_t kSmem2 = sizeof(Smem2) + 1024;
+static_assert(kSmem2 <= 227 * 1024, "shared memory budget");
 
-struct GemmArgs {
+struct Gemm2Args {
   int T, K, N;
   long long out_stride;  // elements
   int silu;
@@ -66,13 +80,90 @@ __device__ __forceinline__ float act(float x, int silu) {
   return fmaf(h, tanh_approx(h), h);
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_bias_act_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tm_x,
-                         const __grid_constant__ CUtensorMap tm_w) {
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// the 256 epilogue threads agree on a flag (barrier 2), so that they leave
+// the tile loop together and never split across named barrier 1
+__device__ __forceinline__ bool epi_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 2, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 2-D TMA load into this CTA's shared memory whose completion counts on the
+// even CTA's barrier at the same offset (no multicast)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar) & kPeerMask), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// arrive on `bar` in both CTAs once every MMA issued so far by this thread completed
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// TMA store of a 2-D box from shared memory (bulk group of this thread)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const Gemm2Args a, const __grid_constant__ CUtensorMap tm_x,
+                     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_out) {
   extern __shared__ uint8_t smem_raw[];
-  GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem2& sm = *reinterpret_cast<Smem2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_m = (a.T + kBM - 1) / kBM, tiles_n = a.N / kBN, n_tiles = tiles_m * tiles_n;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int tiles_m = (a.T + 2 * kBM - 1) / (2 * kBM), tiles_n = a.N / kBN;
+  const int n_units = tiles_m * tiles_n;
   const int nk = a.K / kBK;
 
   if (threadIdx.x == 0) {
@@ -82,95 +173,104 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.acc_full[b], 1);
-      mbar_init(&sm.acc_empty[b], kEpiWarps);
+      mbar_init(&sm.acc_empty[b], 2 * kEpiWarps);
     }
     mbar_init(&sm.done, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, 2 * kAccCols);
-    tmem_relinquish();
+    // both CTAs allocate together (same warp, same destination offset)
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                 "r"(2 * kAccCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_out);
   }
   tc_fence_before();
-  __syncthreads();
+  // barriers of both CTAs are initialised before any CTA touches the other's
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-        const int m0 = (tile / tiles_n) * kBM, n0 = (tile % tiles_n) * kBN;
+      for (int u = pair; ok && u < n_units; u += n_pairs) {
+        const int m0 = (u / tiles_n) * 2 * kBM + rank * kBM;
+        const int n0 = (u % tiles_n) * kBN + rank * (kBN / 2);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kStages;
-          ok = mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, abort_flag, a.hdr, 21);
+          ok = mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, abort_flag, a.hdr, 31);
           if (!ok) break;
-          mbar_arrive_expect_tx(&sm.full[s], kXStage + kWStage);
-          tma_load_2d(sm.x[s], &tm_x, &sm.full[s], kb * kBK, m0);
+          if (leader) mbar_arrive_expect_tx(&sm.full[s], 2 * (kXStage + kWStage));
+          tma_load_2d_pair(sm.x[s], &tm_x, &sm.full[s], kb * kBK, m0);
 #pragma unroll
-          for (int c = 0; c < kBN / 64; ++c)
-            tma_load_2d(sm.w[s] + c * kWChunk, &tm_w, &sm.full[s], n0 + 64 * c, kb * kBK);
+          for (int c = 0; c < kBN / 2 / 64; ++c)
+            tma_load_2d_pair(sm.w[s] + c * kWChunk, &tm_w, &sm.full[s], n0 + 64 * c, kb * kBK);
         }
       }
-      // no copy may still be landing in shared memory when the CTA exits
-      for (int j = max(0, it - kStages); j < it; ++j)
-        mbar_wait(&sm.full[j % kStages], (j / kStages) & 1, nullptr, a.hdr, 29);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, kBN, 0, 1);
+    // ---------------------------------------------------------------- MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16(2 * kBM, kBN, 0, 1);
       int it = 0, tc = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++tc) {
+      for (int u = pair; ok && u < n_units; u += n_pairs, ++tc) {
         const int b = tc & 1;
-        // accumulator b held tile tc - 2 until the epilogue read it
-        ok = mbar_wait(&sm.acc_empty[b], ((tc >> 1) & 1) ^ 1, abort_flag, a.hdr, 22);
+        // accumulator b held tile tc - 2 until both epilogues read it
+        ok = mbar_wait(&sm.acc_empty[b], ((tc >> 1) & 1) ^ 1, abort_flag, a.hdr, 32);
         if (!ok) break;
         tc_fence_after();
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kStages;
-          ok = mbar_wait(&sm.full[s], (it / kStages) & 1, abort_flag, a.hdr, 23);
+          ok = mbar_wait(&sm.full[s], (it / kStages) & 1, abort_flag, a.hdr, 33);
           if (!ok) break;
           tc_fence_after();
           const uint32_t xb = smem_u32(sm.x[s]), wb = smem_u32(sm.w[s]);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_ss(tmem + b * kAccCols, sw128_desc(xb + kk * 32, 16, 1024),
-                   sw128_desc(wb + kk * 16 * 128, kWChunk, 1024), idesc, (kb | kk) != 0);
-          mma_commit(&sm.empty[s]);
+            mma_ss_pair(tmem + b * kAccCols, sw128_desc(xb + kk * 32, 16, 1024),
+                        sw128_desc(wb + kk * 16 * 128, kWChunk, 1024), idesc, (kb | kk) != 0);
+          mma_commit_pair(&sm.empty[s]);
         }
-        if (ok) mma_commit(&sm.acc_full[b]);
+        if (ok) mma_commit_pair(&sm.acc_full[b]);
       }
-      // tensor memory is freed below only after every issued MMA completed
-      mma_commit(&sm.done);
-      mbar_wait(&sm.done, 0, nullptr, a.hdr, 28);
+      // both CTAs learn when every issued MMA completed
+      mma_commit_pair(&sm.done);
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- epilogue
-    const int quarter = warp & 3;  // the TMEM lanes this warp may read
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int quarter = warp & 3;      // the TMEM lanes this warp may read
     const int half = (warp - 2) >> 2;  // columns half*128 .. +127 of the tile
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    // the even CTA's acc_empty barriers, as seen from this CTA
+    const uint32_t empty_addr0 = map_shared(smem_u32(&sm.acc_empty[0]), 0);
+    const uint32_t empty_addr1 = map_shared(smem_u32(&sm.acc_empty[1]), 0);
     int tc = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
+    for (int u = pair; u < n_units; u += n_pairs, ++tc) {
       const int b = tc & 1;
-      const int m0 = (tile / tiles_n) * kBM, n0 = (tile % tiles_n) * kBN;
-      const bool ok = __all_sync(~0u, mbar_wait(&sm.acc_full[b], (tc >> 1) & 1, abort_flag, a.hdr, 24));
+      const bool ok = epi_all(mbar_wait(&sm.acc_full[b], (tc >> 1) & 1, abort_flag, a.hdr, 34));
       if (!ok) break;
       tc_fence_after();
-      const int row = m0 + r;
-      __nv_bfloat16* orow = a.out + (size_t)row * a.out_stride + n0;
+      const int row0 = (u / tiles_n) * 2 * kBM + rank * kBM;
+      const int n0 = (u % tiles_n) * kBN;
+      // the previous tile's TMA stores have read the staging boxes
+      if (tc > 0) {
+        if (warp == 2 && lane == 0) bulk_wait_read();
+        named_bar_sync(1, 32 * kEpiWarps);
+      }
 #pragma unroll 1
       for (int c = half * (kBN / 64); c < (half + 1) * (kBN / 64); ++c) {
         uint32_t acc[32];
@@ -196,23 +296,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(act(__uint_as_float(acc[2 * e]) + bias[2 * e], a.silu),
                               act(__uint_as_float(acc[2 * e + 1]) + bias[2 * e + 1], a.silu));
-        if (row < a.T) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        // the row's 64 bytes of this chunk into box c / 2: 16-byte chunk j of
+        // the box row at j ^ (r & 7) (the TMA store's 128-byte swizzle)
+        const uint32_t box = smem_u32(sm.out[c >> 1]) + r * 128;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        for (int e = 0; e < 4; ++e) {
+          const int j = (c & 1) * 4 + e;
+          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(box + ((j ^ (r & 7)) << 4)), "r"(pk[4 * e]),
+                       "r"(pk[4 * e + 1]), "r"(pk[4 * e + 2]), "r"(pk[4 * e + 3])
+                       : "memory");
         }
       }
-      // this accumulator may take the tile after next
+      // this CTA's part of accumulator b is read: tell the even CTA's issuer
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.acc_empty[b]);
+      if (lane == 0) mbar_arrive_cluster(b ? empty_addr1 : empty_addr0);
+      // the staged tile goes out as four TMA stores (rows past T are dropped)
+      fence_proxy_async_smem();
+      named_bar_sync(1, 32 * kEpiWarps);
+      if (warp == 2 && lane == 0) {
+#pragma unroll
+        for (int bx = 0; bx < kBN / 64; ++bx) tma_store_2d(&tm_out, sm.out[bx], n0 + 64 * bx, row0);
+        bulk_commit();
+      }
     }
+    // the last stores have completed before the CTA's shared memory is released
+    if (warp == 2 && lane == 0) bulk_wait_all();
   }
 
+  // every MMA completed (both CTAs see the commit), then both CTAs meet
+  // before tensor memory is freed and either exits
+  if (warp == 1 && lane == 0) mbar_wait(&sm.done, 0, nullptr, a.hdr, 38);
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 2 * kAccCols);
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kAccCols) : "memory");
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -233,8 +354,7 @@ EncodeTiledFn encode_fn() {
 }
 
 // [rows, cols] bf16 row-major with a row stride: box = box_rows x 64 columns, 128B swizzle
-bool encode_2d(CUtensorMap* m, const void* base, long long rows, long long cols, long long stride,
-               int box_rows) {
+bool encode_2d(CUtensorMap* m, const void* base, long long rows, long long cols, long long stride, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -258,16 +378,18 @@ cudaError_t launch_gemm_sm100(const void* x, long long T, int K, long long x_str
   static int sms[64];
   static unsigned long long attr_set = 0;
   if (!(attr_set & (1ull << dev))) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm_bias_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem2);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     attr_set |= 1ull << dev;
   }
   if (T == 0) return cudaSuccess;
   CUtensorMap tx, tw;
-  if (!encode_2d(&tx, x, T, K, x_stride, kBM) || !encode_2d(&tw, w, K, N, N, kBK)) return cudaErrorInvalidValue;
-  GemmArgs a;
+  CUtensorMap to;
+  if (!encode_2d(&tx, x, T, K, x_stride, kBM) || !encode_2d(&tw, w, K, N, N, kBK) ||
+      !encode_2d(&to, out, T, N, out_stride, kBM))
+    return cudaErrorInvalidValue;
+  Gemm2Args a;
   a.T = (int)T;
   a.K = K;
   a.N = N;
@@ -276,10 +398,21 @@ cudaError_t launch_gemm_sm100(const void* x, long long T, int K, long long x_str
   a.bias = bias;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.hdr = static_cast<WsHeader*>(hdr);
-  const long long tiles = ((T + kBM - 1) / kBM) * (N / kBN);
-  const int grid = (int)std::min<long long>(tiles, sms[dev]);
-  gemm_bias_act_kernel<<<grid, kGemmThreads, kGemmSmem, s>>>(a, tx, tw);
-  return cudaGetLastError();
+  const long long units = ((T + 2 * kBM - 1) / (2 * kBM)) * (N / kBN);
+  const int pairs = (int)std::max<long long>(1, std::min<long long>(units, sms[dev] / 2));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem2;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel, a, tx, tw, to);
 }
 
 }  // namespace hstu

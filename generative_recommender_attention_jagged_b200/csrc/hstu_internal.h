@@ -26,7 +26,8 @@ struct BucketTable {
 };
 
 // Layer glue GEMM on the tensor cores (gemm_sm100.cu): out = act(x W + bias),
-// bf16, K a multiple of 64, N a multiple of 256; hdr = a workspace status header.
+// bf16, on pairs of SMs (tcgen05 cta_group::2) with 256 x 256 output tiles per
+// pair; K a multiple of 64, N a multiple of 256; hdr = a workspace status header.
 bool gemm_sm100_supported(int K, int N);
 cudaError_t launch_gemm_sm100(const void* x, long long T, int K, long long x_stride, const void* w, int N,
                               const float* bias, void* out, long long out_stride, bool silu, void* hdr,

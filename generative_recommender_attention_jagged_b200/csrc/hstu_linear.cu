@@ -201,11 +201,10 @@ int run_linear(const hstu_linear_params* p, const void* x, const void* w, const 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
   char* wsc = static_cast<char*>(ws);
-  // the library's GEMM where its fused epilogue pays: with SiLU (no second pass over
-  // the output) or wide outputs; narrow plain GEMMs (f2) are faster on cuBLASLt
+  // the library's own GEMM (SM pairs, bias and activation in the epilogue) for
+  // every bf16 shape it takes: both projections of the layer
   if (p->dtype == HSTU_DT_BF16 && !(p->flags & HSTU_LIN_CUBLAS) && device_is_sm100(dev) &&
-      hstu::gemm_sm100_supported(p->d_in, p->d_out) && (silu || p->d_out >= 1024)) {
-    // the library's own GEMM: bias and activation in its epilogue
+      hstu::gemm_sm100_supported(p->d_in, p->d_out)) {
     if (cudaMemsetAsync(wsc, 0, kHeaderBytes, stream) != cudaSuccess) return HSTU_ERR_CUDA;
     return hstu::launch_gemm_sm100(x, p->rows, p->d_in, xs, w, p->d_out, bias, out, os, silu, wsc, stream) ==
                    cudaSuccess

@@ -224,11 +224,13 @@ int hstu_ts_bucket(const int64_t* dt, int64_t n, int32_t num_buckets, int32_t* o
  * the four blocks of one [T, 4*H*d] buffer are directly the u, v, q, k
  * arguments of hstu_attn_fwd (token stride 4*H*d).
  *
- * bf16 calls with d_in a multiple of 64, d_out a multiple of 256 and either
- * SiLU (f1) or d_out >= 1024 run the library's own tcgen05 GEMM with the fp32
- * bias and the SiLU in its epilogue (one pass over the output).  Other calls
- * (f2's narrow 512-column output, fp32, HSTU_LIN_CUBLAS) use cuBLASLt (fp32 accumulate, bias in its epilogue) and,
- * for f1, an in-place SiLU kernel.  The first cuBLASLt call on a device
+ * bf16 calls with d_in a multiple of 64 and d_out a multiple of 256 (both
+ * projections of the layer) run the library's own tcgen05 GEMM on pairs of SMs
+ * (256 x 256 output tiles, fp32 accumulate in tensor memory) with the fp32
+ * bias and the SiLU in its epilogue: one pass over the output.  Other calls
+ * (other shapes, fp32, HSTU_LIN_CUBLAS) use cuBLASLt (fp32 accumulate, bias
+ * rounded to bf16 for bf16 calls and added in its epilogue) and, for SiLU, an
+ * in-place SiLU kernel.  The first cuBLASLt call on a device
  * creates that device's handle (host memory owned by cuBLASLt); nothing else
  * is allocated.  The workspace begins with a status word
  * (hstu_check_device_error) that reports a timed-out wait of the GEMM.
@@ -253,8 +255,9 @@ size_t hstu_linear_workspace_size(const hstu_linear_params* p);
 /* out[r, :] = act(x[r, :] W + bias), act = SiLU with HSTU_LIN_SILU, else identity.
  *   x    [rows, d_in]  dtype, row stride x_stride, device, 16-byte aligned
  *   w    [d_in, d_out] dtype, row-major, contiguous, device, 16-byte aligned
- *   bias [d_out] fp32 device or NULL (= 0); for bf16 it is rounded to bf16 into
- *        the workspace and added to the fp32 accumulator in the GEMM epilogue
+ *   bias [d_out] fp32 device or NULL (= 0), added to the fp32 accumulator in the
+ *        GEMM epilogue (on the cuBLASLt route of a bf16 call: rounded to bf16
+ *        into the workspace first)
  *   out  [rows, d_out] dtype, row stride out_stride; must not overlap x or w
  * Returns HSTU_OK, HSTU_ERR_INVALID_ARG / _ALIGNMENT / _WORKSPACE for bad
  * arguments (nothing launched), HSTU_ERR_CUDA if cuBLASLt or a launch fails. */

@@ -110,9 +110,9 @@ def test_whole_layer_matches_oracle():
 
 @pytest.mark.parametrize("T", [1, 300, 4099])
 def test_own_gemm_and_cublas_agree_with_the_oracle(T):
-    """bf16 f1 runs the library's tcgen05 GEMM (bias and SiLU in its epilogue),
-    and so does any wide plain GEMM; the cuBLASLt path must agree within the
-    bf16 tolerance."""
+    """bf16 f1 and f2 both run the library's SM-pair tcgen05 GEMM (bias and
+    SiLU in its epilogue); the cuBLASLt path must agree within the bf16
+    tolerance."""
     w1, b1, w2, b2 = weights(T + 7)
     x = dev(x_rows(T, T + 7))
     z_own = hstu.hstu_layer_f1(x, dev(w1), dev(b1))
@@ -128,6 +128,7 @@ def test_own_gemm_and_cublas_agree_with_the_oracle(T):
     assert rel_err(host64(y_own), y_want) <= BF16_TOL
     assert rel_err(host64(y_lib), y_want) <= BF16_TOL
     assert not torch.equal(z_own, z_lib) or T == 1   # two different kernels ran
+    assert not torch.equal(y_own, y_lib) or T == 1
 
 
 def test_own_gemm_plain_wide_output():
@@ -140,3 +141,20 @@ def test_own_gemm_plain_wide_output():
     want = host64(x) @ host64(w1) + b1
     assert rel_err(host64(own), want) <= BF16_TOL and rel_err(host64(lib), want) <= BF16_TOL
     assert not torch.equal(own, lib)
+
+
+@pytest.mark.parametrize("K,N,silu", [(1024, 1024, True), (1024, 2048, False), (576, 384, True)])
+def test_own_gemm_long_k_schedule(K, N, silu):
+    """Shapes other than the layer's: K = 1024 (16 K-blocks through the 4-stage
+    ring) runs the library's GEMM, a 384-column output (not a multiple of the
+    256-column pair tile) goes to cuBLASLt + the SiLU pass."""
+    T = 1000
+    rng = np.random.default_rng(K + N)
+    x = torch.from_numpy(rng.normal(size=(T, K)).astype(np.float32)).to(torch.bfloat16).cuda()
+    w = torch.from_numpy(rng.uniform(-0.05, 0.05, size=(K, N)).astype(np.float32)).to(torch.bfloat16).cuda()
+    b = torch.from_numpy(rng.normal(0, 0.1, size=N).astype(np.float32)).cuda()
+    got = hstu.hstu_linear(x, w, b, silu=silu)
+    torch.cuda.synchronize()
+    z = host64(x) @ host64(w) + host64(b)
+    want = olayer.silu(z) if silu else z
+    assert rel_err(host64(got), want) <= BF16_TOL
