@@ -854,7 +854,7 @@ def run_glue_bench(args, device):
                          "note": "cuBLASLt GEMM, bias in its epilogue, separate in-place SiLU pass for f1"},
             "roofline": tensor_roofline("gemm_pair_kernel (f1: bias + SiLU in the epilogue)", f1_flops,
                                         *samples["f1"]),
-            "roofline_f2": tensor_roofline("gemm_pair_kernel (f2 = y W2 + b2)", f2_flops, *samples["f2"])}
+            "roofline_f2": tensor_roofline("cuBLASLt GEMM (f2 = y W2 + b2)", f2_flops, *samples["f2"])}
 
 
 def run_mfalcon_bench(args, device):

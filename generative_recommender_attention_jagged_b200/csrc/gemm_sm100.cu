@@ -13,16 +13,23 @@
 // of the next).
 //
 // Roles (320 threads per CTA): warp 0 TMA producer (both CTAs load their own
-// x rows and W half; the bytes complete on the even CTA's barrier), warp 1
-// MMA issuer (even CTA only) and tensor-memory owner (both CTAs allocate
-// collectively), warps 2-9 epilogue (thread = output row, two warps per lane
-// quarter splitting the 256 columns): tcgen05.ld, fp32 bias, SiLU as
-// h + h tanh h with h = x / 2, bf16 into a 128B-swizzled staging tile that
-// one thread stores with TMA (whole 128-byte row segments).  The
-// odd CTA's epilogue frees an accumulator by a remote arrive on the even
-// CTA's barrier.  Every wait is bounded; whatever happens, both CTAs meet at
-// a cluster barrier before tensor memory is freed and the CTAs exit, so
-// neither leaves while the other's MMAs may still read its shared memory.
+// x rows and W half into a 6-stage ring; the bytes complete on the even CTA's
+// barrier), warp 1 MMA issuer (even CTA only) and tensor-memory owner (both
+// CTAs allocate collectively), warps 2-9 epilogue (thread = output row, two
+// warps per lane quarter splitting each 64-column box): tcgen05.ld, fp32
+// bias, SiLU as h + h tanh h with h = x / 2, bf16 into one of two
+// 128B-swizzled staging boxes that one thread stores with TMA (whole
+// 128-byte row segments) while the other box fills.  The odd CTA's epilogue
+// frees an accumulator by a remote arrive on the even CTA's barrier.  Every
+// wait is bounded; whatever happens, both CTAs meet at a cluster barrier
+// before tensor memory is freed and the CTAs exit, so neither leaves while
+// the other's MMAs may still read its shared memory.
+//
+// Measured (T = 53,095 rows, K = 512): steady state is about 42% of the
+// tensor pipe with each SM taking ~26 B/clk of operands from L2, so for a
+// narrow output (N = 512: 5.6 tiles per pair, the last round 62% full) the
+// launch's fill and tail dominate and cuBLASLt is faster; the wide SiLU
+// projection (N = 2048) is about twice as fast as cuBLASLt + a SiLU pass.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -39,7 +46,7 @@ namespace {
 constexpr int kBM = 128;                          // rows per CTA (256 per pair)
 constexpr int kBN = 256;                          // columns per pair tile (128 of W per CTA)
 constexpr int kBK = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kXStage = kBM * kBK * 2;            // 16 KB
 constexpr int kWChunk = kBK * 64 * 2;             // 64 K rows x 64 N columns = 8 KB
 constexpr int kWStage = kWChunk * (kBN / 2 / 64); // this CTA's 128 columns: 16 KB
@@ -53,7 +60,7 @@ constexpr int kOutBox = kBM * 128;               // 128 rows x 64 bf16 columns o
 struct __align__(1024) Smem2 {
   uint8_t x[kStages][kXStage];
   uint8_t w[kStages][kWStage];
-  uint8_t out[kBN / 64][kOutBox];  // this CTA's 128 x 256 bf16 tile, four 128B-swizzled TMA boxes
+  uint8_t out[2][kOutBox];      // two 128B-swizzled TMA boxes (128 rows x 64 columns), used in turn
   uint64_t full[kStages];       // even CTA: both CTAs' bytes of the stage landed
   uint64_t empty[kStages];      // both CTAs: the MMAs that read the stage completed
   uint64_t acc_full[2];         // both CTAs: accumulator b holds a finished tile
@@ -150,7 +157,7 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* s
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -266,13 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int row0 = (u / tiles_n) * 2 * kBM + rank * kBM;
       const int n0 = (u % tiles_n) * kBN;
-      // the previous tile's TMA stores have read the staging boxes
-      if (tc > 0) {
-        if (warp == 2 && lane == 0) bulk_wait_read();
-        named_bar_sync(1, 32 * kEpiWarps);
-      }
+      // box bx (columns 64 bx .. 64 bx + 63) is staged in buffer (4 tc + bx) & 1;
+      // the warps of column half h convert its 32 columns 64 bx + 32 h ..
 #pragma unroll 1
-      for (int c = half * (kBN / 64); c < (half + 1) * (kBN / 64); ++c) {
+      for (int bx = 0; bx < kBN / 64; ++bx) {
+        const int c = 2 * bx + half;  // 32-column chunk of this warp
         uint32_t acc[32];
         tmem_ld32(tmem + lane_base + b * kAccCols + c * 32, acc);
         float bias[32];
@@ -290,34 +295,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) bias[e] = 0.f;
         }
+        // the store issued two boxes ago has read the buffer this box reuses
+        if (tc > 0 || bx >= 2) {
+          if (warp == 2 && lane == 0) bulk_wait_read1();
+          named_bar_sync(1, 32 * kEpiWarps);
+        }
         tmem_wait_ld(acc);
+        if (bx == kBN / 64 - 1) {
+          // this CTA's part of accumulator b is read: tell the even CTA's issuer
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(b ? empty_addr1 : empty_addr0);
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(act(__uint_as_float(acc[2 * e]) + bias[2 * e], a.silu),
                               act(__uint_as_float(acc[2 * e + 1]) + bias[2 * e + 1], a.silu));
-        // the row's 64 bytes of this chunk into box c / 2: 16-byte chunk j of
-        // the box row at j ^ (r & 7) (the TMA store's 128-byte swizzle)
-        const uint32_t box = smem_u32(sm.out[c >> 1]) + r * 128;
+        // the row's 64 bytes into the box: 16-byte chunk j of the box row at
+        // j ^ (r & 7) (the TMA store's 128-byte swizzle)
+        const uint32_t box = smem_u32(sm.out[bx & 1]) + r * 128;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int j = (c & 1) * 4 + e;
+          const int j = half * 4 + e;
           asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(box + ((j ^ (r & 7)) << 4)), "r"(pk[4 * e]),
                        "r"(pk[4 * e + 1]), "r"(pk[4 * e + 2]), "r"(pk[4 * e + 3])
                        : "memory");
         }
-      }
-      // this CTA's part of accumulator b is read: tell the even CTA's issuer
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(b ? empty_addr1 : empty_addr0);
-      // the staged tile goes out as four TMA stores (rows past T are dropped)
-      fence_proxy_async_smem();
-      named_bar_sync(1, 32 * kEpiWarps);
-      if (warp == 2 && lane == 0) {
-#pragma unroll
-        for (int bx = 0; bx < kBN / 64; ++bx) tma_store_2d(&tm_out, sm.out[bx], n0 + 64 * bx, row0);
-        bulk_commit();
+        // the box goes out as one TMA store (rows past T are dropped)
+        fence_proxy_async_smem();
+        named_bar_sync(1, 32 * kEpiWarps);
+        if (warp == 2 && lane == 0) {
+          tma_store_2d(&tm_out, sm.out[bx & 1], n0 + 64 * bx, row0);
+          bulk_commit();
+        }
       }
     }
     // the last stores have completed before the CTA's shared memory is released

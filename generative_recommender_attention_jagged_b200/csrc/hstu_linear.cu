@@ -201,10 +201,12 @@ int run_linear(const hstu_linear_params* p, const void* x, const void* w, const 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
   char* wsc = static_cast<char*>(ws);
-  // the library's own GEMM (SM pairs, bias and activation in the epilogue) for
-  // every bf16 shape it takes: both projections of the layer
+  // the library's own GEMM (SM pairs, bias and activation in the epilogue)
+  // where it is the faster one: SiLU (the activation pass it saves is a full
+  // read + write of the output) or an output of 1024+ columns; a narrow plain
+  // projection (f2) has too few output tiles per SM pair and goes to cuBLASLt
   if (p->dtype == HSTU_DT_BF16 && !(p->flags & HSTU_LIN_CUBLAS) && device_is_sm100(dev) &&
-      hstu::gemm_sm100_supported(p->d_in, p->d_out)) {
+      hstu::gemm_sm100_supported(p->d_in, p->d_out) && (silu || p->d_out >= 1024)) {
     if (cudaMemsetAsync(wsc, 0, kHeaderBytes, stream) != cudaSuccess) return HSTU_ERR_CUDA;
     return hstu::launch_gemm_sm100(x, p->rows, p->d_in, xs, w, p->d_out, bias, out, os, silu, wsc, stream) ==
                    cudaSuccess

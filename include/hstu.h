@@ -224,11 +224,12 @@ int hstu_ts_bucket(const int64_t* dt, int64_t n, int32_t num_buckets, int32_t* o
  * the four blocks of one [T, 4*H*d] buffer are directly the u, v, q, k
  * arguments of hstu_attn_fwd (token stride 4*H*d).
  *
- * bf16 calls with d_in a multiple of 64 and d_out a multiple of 256 (both
- * projections of the layer) run the library's own tcgen05 GEMM on pairs of SMs
- * (256 x 256 output tiles, fp32 accumulate in tensor memory) with the fp32
- * bias and the SiLU in its epilogue: one pass over the output.  Other calls
- * (other shapes, fp32, HSTU_LIN_CUBLAS) use cuBLASLt (fp32 accumulate, bias
+ * bf16 calls with d_in a multiple of 64, d_out a multiple of 256 and either
+ * SiLU (f1) or d_out >= 1024 run the library's own tcgen05 GEMM on pairs of
+ * SMs (256 x 256 output tiles, fp32 accumulate in tensor memory) with the
+ * fp32 bias and the SiLU in its epilogue: one pass over the output.  Other
+ * calls (f2's narrow 512-column output, where cuBLASLt is faster; other
+ * shapes, fp32, HSTU_LIN_CUBLAS) use cuBLASLt (fp32 accumulate, bias
  * rounded to bf16 for bf16 calls and added in its epilogue) and, for SiLU, an
  * in-place SiLU kernel.  The first cuBLASLt call on a device
  * creates that device's handle (host memory owned by cuBLASLt); nothing else

@@ -110,9 +110,9 @@ def test_whole_layer_matches_oracle():
 
 @pytest.mark.parametrize("T", [1, 300, 4099])
 def test_own_gemm_and_cublas_agree_with_the_oracle(T):
-    """bf16 f1 and f2 both run the library's SM-pair tcgen05 GEMM (bias and
-    SiLU in its epilogue); the cuBLASLt path must agree within the bf16
-    tolerance."""
+    """bf16 f1 runs the library's SM-pair tcgen05 GEMM (bias and SiLU in its
+    epilogue), f2 (512 columns) cuBLASLt; both routes must agree with the
+    oracle within the bf16 tolerance."""
     w1, b1, w2, b2 = weights(T + 7)
     x = dev(x_rows(T, T + 7))
     z_own = hstu.hstu_layer_f1(x, dev(w1), dev(b1))
@@ -128,7 +128,6 @@ def test_own_gemm_and_cublas_agree_with_the_oracle(T):
     assert rel_err(host64(y_own), y_want) <= BF16_TOL
     assert rel_err(host64(y_lib), y_want) <= BF16_TOL
     assert not torch.equal(z_own, z_lib) or T == 1   # two different kernels ran
-    assert not torch.equal(y_own, y_lib) or T == 1
 
 
 def test_own_gemm_plain_wide_output():
@@ -145,7 +144,7 @@ def test_own_gemm_plain_wide_output():
 
 @pytest.mark.parametrize("K,N,silu", [(1024, 1024, True), (1024, 2048, False), (576, 384, True)])
 def test_own_gemm_long_k_schedule(K, N, silu):
-    """Shapes other than the layer's: K = 1024 (16 K-blocks through the 4-stage
+    """Shapes other than the layer's: K = 1024 (16 K-blocks through the 6-stage
     ring) runs the library's GEMM, a 384-column output (not a multiple of the
     256-column pair tile) goes to cuBLASLt + the SiLU pass."""
     T = 1000
