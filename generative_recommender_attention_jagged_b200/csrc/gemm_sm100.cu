@@ -23,13 +23,16 @@
 // frees an accumulator by a remote arrive on the even CTA's barrier.  Every
 // wait is bounded; whatever happens, both CTAs meet at a cluster barrier
 // before tensor memory is freed and the CTAs exit, so neither leaves while
-// the other's MMAs may still read its shared memory.
+// the other's MMAs may still read its shared memory or copies into it are in
+// flight.
 //
-// Measured (T = 53,095 rows, K = 512): steady state is about 42% of the
-// tensor pipe with each SM taking ~26 B/clk of operands from L2, so for a
-// narrow output (N = 512: 5.6 tiles per pair, the last round 62% full) the
-// launch's fill and tail dominate and cuBLASLt is faster; the wide SiLU
-// projection (N = 2048) is about twice as fast as cuBLASLt + a SiLU pass.
+// Measured (T = 53,095 rows, K = 512): the wide SiLU projection (N = 2048)
+// at about two thirds of the measured bf16 peak, twice as fast as cuBLASLt + a
+// SiLU pass.  A narrow output (N = 512: 5.6 tiles per pair, the last round 62%
+// full) is dominated by the launch's fill and tail, where cuBLASLt is faster.
+//
+// The remote arrive and every wait use CTA scope (a cluster-scope release or
+// acquire costs a memory barrier per use: 10% of this kernel's time).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -37,8 +40,8 @@
 #include <cstdint>
 #include <mutex>
 
-#include "device_common.cuh"
 #include "hstu_internal.h"
+#include "pair_common.cuh"
 
 namespace hstu {
 namespace {
@@ -53,7 +56,6 @@ constexpr int kWStage = kWChunk * (kBN / 2 / 64); // this CTA's 128 columns: 16 
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr uint32_t kAccCols = kBN;                // one fp32 accumulator: 256 columns
-constexpr uint32_t kPeerMask = 0xFEFFFFFFu;       // clears the CTA-rank bit of a shared::cluster address
 
 constexpr int kOutBox = kBM * 128;               // 128 rows x 64 bf16 columns of output: 16 KB
 
@@ -68,6 +70,7 @@ struct __align__(1024) Smem2 {
   uint64_t done;                // both CTAs: every MMA completed
   uint32_t tmem_base;
   int abort;
+  int issued;                   // stages whose copies this CTA issued
 };
 constexpr size_t kSmem2 = sizeof(Smem2) + 1024;
 static_assert(kSmem2 <= 227 * 1024, "shared memory budget");
@@ -87,23 +90,6 @@ __device__ __forceinline__ float act(float x, int silu) {
   return fmaf(h, tanh_approx(h), h);
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// address of the same shared variable in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t map_shared(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
 // the 256 epilogue threads agree on a flag (barrier 2), so that they leave
 // the tile loop together and never split across named barrier 1
 __device__ __forceinline__ bool epi_all(bool ok) {
@@ -115,38 +101,6 @@ __device__ __forceinline__ bool epi_all(bool ok) {
       : "r"((uint32_t)ok)
       : "memory");
   return r != 0;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// 2-D TMA load into this CTA's shared memory whose completion counts on the
-// even CTA's barrier at the same offset (no multicast)
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar) & kPeerMask), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// arrive on `bar` in both CTAs once every MMA issued so far by this thread completed
-__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
-          smem_u32(bar))
-      : "memory");
 }
 
 // TMA store of a 2-D box from shared memory (bulk group of this thread)
@@ -184,14 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sm.done, 1);
     sm.abort = 0;
+    sm.issued = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
     // both CTAs allocate together (same warp, same destination offset)
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
-                 "r"(2 * kAccCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    tmem_alloc_pair(&sm.tmem_base, 2 * kAccCols);
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_x);
@@ -222,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < kBN / 2 / 64; ++c)
             tma_load_2d_pair(sm.w[s] + c * kWChunk, &tm_w, &sm.full[s], n0 + 64 * c, kb * kBK);
+          sm.issued = it + 1;
         }
       }
     }
@@ -305,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // this CTA's part of accumulator b is read: tell the even CTA's issuer
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(b ? empty_addr1 : empty_addr0);
+          if (lane == 0) mbar_arrive_remote(b ? empty_addr1 : empty_addr0);
         }
         uint32_t pk[16];
 #pragma unroll
@@ -335,16 +288,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 2 && lane == 0) bulk_wait_all();
   }
 
-  // every MMA completed (both CTAs see the commit), then both CTAs meet
-  // before tensor memory is freed and either exits
+  // Every MMA completed (both CTAs see the commit) and both CTAs meet, the
+  // issued counts published; the even CTA then accounts for every copy into
+  // either CTA (a stage expected but not issued by the odd CTA, or issued but
+  // not expected, which only a timed-out wait leaves behind), and both meet
+  // again before tensor memory is freed and either exits, so no copy lands
+  // in a CTA that has left.
   if (warp == 1 && lane == 0) mbar_wait(&sm.done, 0, nullptr, a.hdr, 38);
   __syncwarp();
   tc_fence_before();
   __syncthreads();
   cluster_sync();
+  if (leader && warp == 0 && lane == 0) {
+    const int mine = sm.issued;
+    const int peer = (int)ld_shared_cluster_u32(map_shared(smem_u32(&sm.issued), 1));
+    const int last = max(mine, peer);
+    for (int t = max(0, last - kStages); t < last; ++t) {
+      uint64_t* bar = &sm.full[t % kStages];
+      if (t < mine && t >= peer) mbar_complete_tx(bar, kXStage + kWStage);       // odd half never issued
+      if (t >= mine && t < peer) mbar_arrive_expect_tx(bar, kXStage + kWStage);  // odd half never expected
+      mbar_wait(bar, (t / kStages) & 1, nullptr, a.hdr, 39);
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   if (warp == 1)
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kAccCols) : "memory");
+    tmem_dealloc_pair(tmem, 2 * kAccCols);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
