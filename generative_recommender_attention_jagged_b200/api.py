@@ -380,9 +380,11 @@ def hstu_mfalcon_fwd(q_c, k_c, v_c, u_c, cand_offsets, hist_timestamps, hist_ts_
 
 def hstu_attn_bwd(q, k, v, seq_offsets, timestamps, rab_pos, rab_ts, d_o, *, n_max: int,
                   alpha: Optional[float] = None, num_candidates=None, max_seq_len: Optional[int] = None,
-                  workspace=None, stream=None):
+                  workspace=None, stream=None, force_simt: bool = False):
     """Gradients of the raw per-head output o = A V: returns d_q, d_k, d_v [T, H, d]
-    and d_rab_pos, d_rab_ts (all fp32)."""
+    and d_rab_pos, d_rab_ts (all fp32).  bf16 inputs with d = 128 run on the
+    tensor cores (bf16 GEMM operands); force_simt keeps them on the fp32
+    CUDA-core kernel."""
     T, H, d = q.shape
     dt = q.dtype
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -400,7 +402,8 @@ def hstu_attn_bwd(q, k, v, seq_offsets, timestamps, rab_pos, rab_ts, d_o, *, n_m
         raise ValueError("q, k and v must share one token stride")
     params = attn_params(batch=seq_offsets.numel() - 1, num_heads=H, head_dim=d, n_max=n_max, total_tokens=T,
                          max_seq_len=n_max if max_seq_len is None else max_seq_len, dtype=dt, alpha=alpha,
-                         num_ts_buckets=rab_ts.numel(), qkv_stride=qs)
+                         num_ts_buckets=rab_ts.numel(), qkv_stride=qs,
+                         flags=_lib.F_FORCE_SIMT if force_simt else 0)
     grads = [torch.empty(T, H, d, dtype=torch.float32, device=q.device) for _ in range(3)]
     d_rp = torch.empty_like(rab_pos)
     d_rt = torch.empty_like(rab_ts)

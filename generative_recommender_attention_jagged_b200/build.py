@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhstu.so")
-SOURCES = ["hstu_api.cpp", "ts_table.cpp", "hstu_kernels.cu", "attn_sm100.cu", "attn_sm100_single.cu", "hstu_static_ws.cu", "hstu_linear.cu", "hstu_kv.cu", "hstu_mfalcon.cu", "gemm_sm100.cu", "hstu_bwd.cu"]
+SOURCES = ["hstu_api.cpp", "ts_table.cpp", "hstu_kernels.cu", "attn_sm100.cu", "attn_sm100_single.cu", "hstu_static_ws.cu", "hstu_linear.cu", "hstu_kv.cu", "hstu_mfalcon.cu", "gemm_sm100.cu", "hstu_bwd.cu", "attn_bwd_sm100.cu"]
 HEADERS = ["hstu_internal.h", "device_common.cuh", "attn_common.cuh", "pair_common.cuh"]
 
 

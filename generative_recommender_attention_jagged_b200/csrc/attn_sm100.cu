@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int item_idx = blockIdx.x;
   if (item_idx >= a.hdr->n_items) return;
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& sm = aligned_smem<Smem>(smem_raw);
 
   const WorkItem it = a.items[item_idx];
   // a work list not written by this call's scheduler must not send us out of bounds

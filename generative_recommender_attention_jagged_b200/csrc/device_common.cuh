@@ -110,6 +110,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The 1024-byte aligned start of the dynamic shared memory, derived from the
+// __shared__ array by pointer arithmetic so that the compiler keeps the shared
+// address space (a round trip through an integer turns every access through
+// the result into a generic one: generic atomics and loads take the L1TEX
+// path instead of the shared-memory pipe).
+template <typename T>
+__device__ __forceinline__ T& aligned_smem(uint8_t* smem_raw) {
+  return *reinterpret_cast<T*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }

@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const Gemm2Args a, const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_out) {
   extern __shared__ uint8_t smem_raw[];
-  Smem2& sm = *reinterpret_cast<Smem2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem2& sm = aligned_smem<Smem2>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;

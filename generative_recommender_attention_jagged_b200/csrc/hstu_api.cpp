@@ -347,8 +347,19 @@ int hstu_attn_fwd_paged(const hstu_attn_params* p, const void* q_new, const void
   return run(p, c);
 }
 
+// the tensor-core backward applies: bf16, d = 128, sm_100, not forced onto CUDA cores
+bool bwd_on_tensor_cores(const hstu_attn_params* p) {
+  return p->dtype == HSTU_DT_BF16 && p->head_dim == 128 && !(p->flags & HSTU_F_FORCE_SIMT) && device_is_sm100();
+}
+
+// bytes of the bf16 copy of d_o the tensor-core backward stages after the status header
+size_t bwd_g_bytes(const hstu_attn_params* p) {
+  return bwd_on_tensor_cores(p) ? (size_t)p->total_tokens * p->num_heads * p->head_dim * 2 : 0;
+}
+
 size_t hstu_attn_bwd_workspace_size(const hstu_attn_params* p) {
-  return check_params(p) == HSTU_OK ? sizeof(WsHeader) : 0;
+  if (check_params(p) != HSTU_OK) return 0;
+  return align_up(sizeof(WsHeader)) + bwd_g_bytes(p);
 }
 
 int hstu_attn_bwd(const hstu_attn_params* p, const void* q, const void* k, const void* v,
@@ -365,7 +376,9 @@ int hstu_attn_bwd(const hstu_attn_params* p, const void* q, const void* k, const
   const void* ptrs[] = {q, k, v, d_o, d_q, d_k, d_v, workspace};
   for (const void* ptr : ptrs)
     if (ptr && !aligned16(ptr)) return HSTU_ERR_ALIGNMENT;
-  if (workspace_bytes < sizeof(WsHeader)) return HSTU_ERR_WORKSPACE;
+  const size_t g_bytes = bwd_g_bytes(p);
+  if (workspace_bytes < sizeof(WsHeader) || (g_bytes && workspace_bytes < align_up(sizeof(WsHeader)) + g_bytes))
+    return HSTU_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   AttnArgs a;
   std::memset(&a, 0, sizeof a);
@@ -398,6 +411,17 @@ int hstu_attn_bwd(const hstu_attn_params* p, const void* q, const void* k, const
   // the forward's checks of offsets, lengths, candidate counts and timestamps
   if (launch_plan(a, false, p->max_seq_len, s) != cudaSuccess) return HSTU_ERR_CUDA;
   const BucketTable& thr = bucket_table(a.nb);
+  if (g_bytes) {
+    void* g = static_cast<char*>(workspace) + align_up(sizeof(WsHeader));
+    CUtensorMap tq, tk, tv, tg;
+    if (!encode_rows(&tq, q, a.T_q, a.H, a.d, a.qkv_stride) || !encode_rows(&tk, k, a.T_q, a.H, a.d, a.qkv_stride) ||
+        !encode_rows(&tv, v, a.T_q, a.H, a.d, a.qkv_stride) || !encode_rows(&tg, g, a.T_q, a.H, a.d, a.H * a.d))
+      return HSTU_ERR_CUDA;
+    return launch_attn_bwd_sm100(a, thr, d_o, g, tq, tk, tv, tg, d_q, d_k, d_v, d_rab_pos, d_rab_ts, s) ==
+                   cudaSuccess
+               ? HSTU_OK
+               : HSTU_ERR_CUDA;
+  }
   return launch_attn_bwd(a, thr, d_o, d_q, d_k, d_v, d_rab_pos, d_rab_ts, s) == cudaSuccess ? HSTU_OK
                                                                                             : HSTU_ERR_CUDA;
 }

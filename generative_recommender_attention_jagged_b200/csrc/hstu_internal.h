@@ -131,6 +131,13 @@ cudaError_t launch_attn_simt(const AttnArgs& a, const BucketTable& thr, cudaStre
 // d_rp / d_rt must be zeroed by the caller.
 cudaError_t launch_attn_bwd(const AttnArgs& a, const BucketTable& thr, const float* d_o, float* dq, float* dk,
                             float* dv, float* d_rp, float* d_rt, cudaStream_t s);
+// Backward on the tensor cores (attn_bwd_sm100.cu): bf16 inputs, d = 128.
+// g_bf16: scratch for d_o rounded to bf16 ([T, H, 128]); tm_g maps it.
+bool attn_bwd_sm100_supported(const AttnArgs& a);
+cudaError_t launch_attn_bwd_sm100(const AttnArgs& a, const BucketTable& thr, const float* d_o, void* g_bf16,
+                                  const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                  const CUtensorMap& tm_g, float* dq, float* dk, float* dv, float* d_rp,
+                                  float* d_rt, cudaStream_t s);
 cudaError_t launch_epilogue(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_ts_bucket(const int64_t* dt, int64_t n, int32_t* out, const BucketTable& thr,
                              cudaStream_t s);

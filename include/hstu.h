@@ -285,11 +285,18 @@ int hstu_layer_f2(const hstu_linear_params* p, const void* y, const void* w2, co
  *   d_q_i = alpha sum_j ds_ij k_j,   d_k_j = alpha sum_i ds_ij q_i,
  *   d_v_j = sum_i a_ij d_o_i,        d_rab_pos[p(i)-p(j)+n_max-1] += ds_ij,
  *   d_rab_ts[b(i,j)] += ds_ij
- * Computed on CUDA cores in fp32 (scores recomputed as in the forward).
+ * bf16 inputs with d = 128 run on the tensor cores (tcgen05): d_o is rounded
+ * to bf16 into the workspace, the weights a and the score gradients ds are
+ * rounded to bf16 as GEMM operands, all sums accumulate in fp32 (the bf16
+ * tolerance of the forward applies).  Other inputs, or HSTU_F_FORCE_SIMT in
+ * p->flags, run on CUDA cores in fp32.  Scores are recomputed as in the
+ * forward (exact time buckets).
  *   q, k, v     [T, H, d] dtype with token stride p->qkv_stride
  *   d_o         [T, H, d] fp32 contiguous
  *   d_q, d_k, d_v [T, H, d] fp32 contiguous (written)
  *   d_rab_pos   [2*n_max-1] fp32, d_rab_ts [num_ts_buckets] fp32 (zeroed, then summed)
+ *   workspace   hstu_attn_bwd_workspace_size(p) bytes: the status header and,
+ *               on the tensor-core path, T*H*d*2 bytes for the bf16 copy of d_o
  * With T = 0 the arrays indexed by token may be NULL (the bias-table
  * gradients are still zeroed).
  * Device checks as in hstu_attn_fwd (status word in the workspace).
