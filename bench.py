@@ -44,8 +44,8 @@ TILE = 128
 #   ncu --set full --clock-control none -k regex:attn_sm100_single -s 10 -c 1 \
 #       python bench.py --only paged --steps 3 --warmup 3
 # None whenever the kernel has changed since its counters were taken.
-ATTN_TRAFFIC_BYTES = 406_045_696 + 76_942_848
-PAGED_TRAFFIC_BYTES = 115_100_672 + 5_167_104
+ATTN_TRAFFIC_BYTES = 401_281_280 + 75_198_720
+PAGED_TRAFFIC_BYTES = 114_908_672 + 4_225_024
 
 
 def allowed_pairs(lengths, cands=None):
