@@ -456,7 +456,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile when the other has some) issued no GEMM, so nothing waited for its
     // Q copy; that copy lands in the staging area used below
     if (ok && cnt == 0 && exists) ok = ew_all(mbar_wait(&sm.bar_q, 0, abort_flag, a.hdr, 7), group);
-    if (ok && exists) {
+    if (ok && exists && a.o_bf16) {
+      // O of this warpgroup's 64 columns as bf16 (one split feeding the
+      // LayerNorm gate): 128 rows x 128 bytes staged in its half of the tile's
+      // Q buffer, 16-byte chunk c of row r at c ^ (r & 7), then whole 128-byte
+      // row segments per warp
+      const uint32_t stage = smem_u32(sm.q[x]) + half * (kTileBytes / 2);
+      const int wq = warp & 3;
+      uint32_t pk[32];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t orr[32];
+        if (cnt > 0) {
+          tmem_ld32(tmem + lane_base + 256 + x * 128 + half * 64 + h2 * 32, orr);
+          tmem_wait_ld(orr);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[e] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[16 * h2 + e] = pack_bf16x2(__uint_as_float(orr[2 * e]), __uint_as_float(orr[2 * e + 1]));
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        sts_v4(stage + r * 128 + ((c ^ (r & 7)) << 4), make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+      named_bar_sync(1 + group, kTile);
+#pragma unroll 1
+      for (int rr = 4 * wq + (lane >> 3); rr < kTile; rr += 16) {
+        const int c = lane & 7;
+        if (rr < g.nq_rows) {
+          const uint4 val = lds_v4(stage + rr * 128 + ((c ^ (rr & 7)) << 4));
+          __nv_bfloat16* orow =
+              reinterpret_cast<__nv_bfloat16*>(a.o_ws) + ((size_t)(g.qrow0 + rr) * a.H + it.head) * kHeadDim;
+          *reinterpret_cast<uint4*>(orow + half * 64 + 8 * c) = val;
+        }
+      }
+    } else if (ok && exists) {
       // O of this warpgroup's 64 columns goes out through shared memory, 32
       // columns at a time: its half of the tile's Q buffer (free once the
       // tile's GEMMs completed) holds 128 rows x 128 bytes, 16-byte chunk c of

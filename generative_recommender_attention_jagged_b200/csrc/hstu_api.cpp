@@ -197,6 +197,12 @@ int run(const hstu_attn_params* p, const Common& c) {
   a.max_items = l.max_items;
   a.item_tiles = item_tiles;
   a.out_raw = (p->flags & HSTU_F_OUTPUT_RAW_AV) ? 1 : 0;
+  // one split of A.V partials feeding the LayerNorm gate is rounded to bf16
+  // once (y is bf16 and normalised right after): half the bytes written and read
+  a.o_bf16 = (tc && item_tiles == 2 && !c.paged && a.num_splits == 1 && !a.out_raw &&
+              (p->num_heads * p->head_dim) % 128 == 0)
+                 ? 1
+                 : 0;
   a.self_term = tc ? 1 : 0;
   a.out_bf16 = p->dtype == HSTU_DT_BF16 ? 1 : 0;
   a.in_bf16 = p->dtype == HSTU_DT_BF16 ? 1 : 0;

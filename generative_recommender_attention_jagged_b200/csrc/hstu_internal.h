@@ -72,6 +72,7 @@ struct AttnArgs {
   int32_t out_bf16;     // out dtype
   int32_t in_bf16;      // q/k/v/u/pool dtype
   int32_t precise_silu; // tensor-core path: fp32 tanh per score instead of packed bf16x2
+  int32_t o_bf16;       // o_ws holds one split of bf16 partials (two-tile kernel, y output)
   const void* q;
   const void* k;
   const void* v;

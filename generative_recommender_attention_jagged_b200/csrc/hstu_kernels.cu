@@ -436,8 +436,21 @@ __global__ void __launch_bounds__(256) epilogue_vec_kernel(const AttnArgs a) {
       }
     }
     float o[VPT][4];
+    if (a.o_bf16) {  // one split of bf16 partials
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) {
+      for (int k = 0; k < VPT; ++k) {
+        const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.o_ws) +
+                                                                (size_t)row * D + 128 * k + 4 * lane));
+        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+        o[k][0] = __low2float(lo);
+        o[k][1] = __high2float(lo);
+        o[k][2] = __low2float(hi);
+        o[k][3] = __high2float(hi);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < VPT && !a.o_bf16; ++k) {
       const float4* src = reinterpret_cast<const float4*>(a.o_ws + (size_t)row * D + 128 * k + 4 * lane);
       float4 acc = __ldcs(src);
       for (int sp = 1; sp < a.num_splits; ++sp) {
