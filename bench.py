@@ -44,7 +44,7 @@ TILE = 128
 #   ncu --set full --clock-control none -k regex:attn_sm100_single -s 10 -c 1 \
 #       python bench.py --only paged --steps 3 --warmup 3
 # None whenever the kernel has changed since its counters were taken.
-ATTN_TRAFFIC_BYTES = 401_281_280 + 75_198_720
+ATTN_TRAFFIC_BYTES = 394_607_616 + 36_452_352
 PAGED_TRAFFIC_BYTES = 114_908_672 + 4_225_024
 
 
