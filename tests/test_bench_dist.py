@@ -54,3 +54,18 @@ def test_rank_seeds():
 
 def test_single_rank_needs_no_process_group():
     assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
+
+
+def test_peak_follows_the_clock_the_region_ran_at():
+    """The burst bf16 peak applies whenever the median SM clock held within 5%
+    of its maximum, power-cap flags or not; a region the cap slowed takes the
+    sustained peak; both fractions are reported by tensor_roofline."""
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    hot = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped_hot = {"sm_mhz": 1942.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    slowed = {"sm_mhz": 1342.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.pick_bf16_peak(peaks, hot)[0] == 1600.0
+    assert bench.pick_bf16_peak(peaks, capped_hot)[0] == 1600.0
+    assert "sw_power_cap seen" in bench.pick_bf16_peak(peaks, capped_hot)[1]
+    assert bench.pick_bf16_peak(peaks, slowed)[0] == 1400.0
+    assert bench.pick_bf16_peak(peaks, None)[0] == 1600.0
